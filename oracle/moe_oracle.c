@@ -1,0 +1,391 @@
+/*
+ * moe_oracle.c -- plain, slow CPU oracle for MoE token dispatch and combine.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the checker, not the product: only
+ * the test suite, the package's smoke check and the benchmark's CPU-baseline
+ * leg may load it.  It shares no code, header, table or constant with the
+ * CUDA library; the status bit values below are this file's own copy of the
+ * documented contract.
+ *
+ * Every routine is single-threaded, uses plain loops, and does its floating
+ * point in fp64 unless a rounding step is part of the definition.  Sources:
+ *
+ *  [DeepEP-272]  DeepEP issue "Does Deepep's Dispatch/Combine Support Autograd
+ *                Like PyTorch's all_to_all?" -- get_dispatch_layout outputs
+ *                (num_tokens_per_rank, num_tokens_per_expert,
+ *                is_token_in_rank); dispatch backward is a combine.
+ *  [DS-8847]     DeepSpeed PR "AutoEP: support combine_impl=fused_weighted_sum
+ *                with AutoEP+AutoTP folding", sections Problem / Change /
+ *                Benchmark -- flat index token*top_k+slot, router-dtype
+ *                weights scattered to [tokens, top_k], FP32 accumulation,
+ *                coverage RuntimeError, row and score gradients.
+ *  [DS-AutoEP]   DeepSpeed AutoEP base PR, sections Attribution and Design --
+ *                reorder tokens by expert, token-group alignment / padding
+ *                for grouped GEMM, restore the original token order.
+ *  [DS-8190]     DeepSpeed PR "Derive AutoEP rank splits from the per-expert
+ *                count exchange", sections Redundancy and Fix -- the count
+ *                matrix [ep_size, E_local], input_splits = its row sums, and
+ *                received_counts.sum(dim=1) == output_splits.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - padding: an expert with c tokens occupies ceil(c/align)*align rows, so an
+ *    empty expert occupies none;
+ *  - order inside an expert's group: stable by flat index (token, then slot);
+ *  - logical ranks: source rank s owns tokens [s*T/R, (s+1)*T/R), destination
+ *    rank r owns experts [r*E/R, (r+1)*E/R);
+ *  - an out-of-range expert id (including -1) is an error: the assignment is
+ *    skipped and the EXPERT_OOR bit is returned;
+ *  - pad rows are zero, rows past the padded total are left untouched and
+ *    carry row_to_flat = -1;
+ *  - the FP32 combine is an fmaf chain over slots k = 0..K-1 from 0 with one
+ *    round-to-nearest-even to bf16 (reported by out_seq); the fp64 sum is the
+ *    reference value the tolerance is measured against;
+ *  - grad_w is accumulated in fp64 (bf16 x bf16 products are exact).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Status bits (the library's documented values; this file's own copy). */
+#define ORC_EXPERT_OOR 1
+#define ORC_CAPACITY 2
+#define ORC_ROW_OOR 4
+#define ORC_COVERAGE 8
+
+/* ---------------------------------------------------------------- bf16 --- */
+
+/* bfloat16 is the top 16 bits of an IEEE binary32.  Round to nearest, ties to
+ * even, from the definition: keep the top half; look at the discarded low
+ * half; above the midpoint round up, below it keep, exactly at it round up
+ * only when the kept value is odd.  Rounding up is +1 on the kept bits, which
+ * carries into the exponent (and to infinity) as IEEE ordering requires.
+ * NaN stays NaN (quiet bit forced). */
+uint16_t oracle_bf16_from_float(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t kept = u >> 16;
+    uint32_t low = u & 0xffffu;
+    if (low > 0x8000u || (low == 0x8000u && (kept & 1u))) kept += 1u;
+    return (uint16_t)kept;
+}
+
+float oracle_float_from_bf16(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Element-wise helpers so tests can pin the rounding against a library. */
+void oracle_bf16_round_array(const float* in, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_from_float(in[i]);
+}
+
+/* -------------------------------------------------------------- layout --- */
+
+/* get_dispatch_layout [DeepEP-272] plus the count matrix of [DS-8190] and the
+ * padded group offsets of [DS-AutoEP] (alignment / padding helpers).
+ *
+ *   tokens_per_expert[e]        = #{(t,k) : topk_idx[t,k] = e}
+ *   counts[s][r][el]            = #{(t,k) : t in block s, topk_idx[t,k] = r*El+el}
+ *   splits[s][r]                = sum over el of counts[s][r][el]
+ *                                 (row s = input_splits of source rank s)
+ *   is_token_in_rank[t][r]      = 1 if some slot of t routes to an expert of r
+ *   tokens_per_rank[s][r]       = #{t in block s : is_token_in_rank[t][r]}
+ *   offsets[0] = 0, offsets[e+1] = offsets[e] + ceil(c_e/align)*align
+ *
+ * Returns status bits (ORC_EXPERT_OOR if some id is outside [0, E)). */
+int oracle_layout(const int64_t* topk_idx, int T, int K, int E, int R, int align,
+                  int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                  int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
+                  int32_t* offsets) {
+    int status = 0;
+    int El = E / R;
+    int Tb = T / R;
+    memset(tokens_per_expert, 0, sizeof(int32_t) * (size_t)E);
+    memset(counts, 0, sizeof(int32_t) * (size_t)R * (size_t)E);
+    memset(splits, 0, sizeof(int32_t) * (size_t)R * (size_t)R);
+    memset(tokens_per_rank, 0, sizeof(int32_t) * (size_t)R * (size_t)R);
+    memset(is_token_in_rank, 0, (size_t)T * (size_t)R);
+
+    for (int t = 0; t < T; ++t) {
+        int s = t / Tb;
+        for (int k = 0; k < K; ++k) {
+            int64_t e = topk_idx[(int64_t)t * K + k];
+            if (e < 0 || e >= E) {
+                status |= ORC_EXPERT_OOR;
+                continue;
+            }
+            int r = (int)(e / El);
+            int el = (int)(e % El);
+            tokens_per_expert[e] += 1;
+            counts[((int64_t)s * R + r) * El + el] += 1;
+            is_token_in_rank[(int64_t)t * R + r] = 1;
+        }
+    }
+    for (int s = 0; s < R; ++s)
+        for (int r = 0; r < R; ++r) {
+            int32_t sum = 0;
+            for (int el = 0; el < El; ++el) sum += counts[((int64_t)s * R + r) * El + el];
+            splits[s * R + r] = sum;
+        }
+    for (int t = 0; t < T; ++t) {
+        int s = t / Tb;
+        for (int r = 0; r < R; ++r) tokens_per_rank[s * R + r] += is_token_in_rank[(int64_t)t * R + r];
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) {
+        int32_t c = tokens_per_expert[e];
+        int32_t padded = ((c + align - 1) / align) * align;
+        offsets[e + 1] = offsets[e] + padded;
+    }
+    return status;
+}
+
+/* output_splits of every destination rank, counted directly: the number of
+ * assignments source block s sends to rank r, i.e. what the per-rank-total
+ * exchange of [DS-8190] (Redundancy, "exchange 1") would have delivered.
+ * Independent of the count matrix, so that received_counts.sum(dim=1) ==
+ * output_splits can be checked against it.  out[r][s]. */
+void oracle_output_splits(const int64_t* topk_idx, int T, int K, int E, int R, int32_t* out) {
+    int El = E / R;
+    int Tb = T / R;
+    for (int r = 0; r < R; ++r)
+        for (int s = 0; s < R; ++s) {
+            int32_t n = 0;
+            for (int t = s * Tb; t < (s + 1) * Tb; ++t)
+                for (int k = 0; k < K; ++k) {
+                    int64_t e = topk_idx[(int64_t)t * K + k];
+                    if (e >= (int64_t)r * El && e < (int64_t)(r + 1) * El) ++n;
+                }
+            out[r * R + s] = n;
+        }
+}
+
+/* ------------------------------------------------------------- permute --- */
+
+typedef struct {
+    int32_t expert;
+    int32_t flat;
+} orc_assign;
+
+static int orc_cmp_assign(const void* a, const void* b) {
+    const orc_assign* x = (const orc_assign*)a;
+    const orc_assign* y = (const orc_assign*)b;
+    if (x->expert != y->expert) return x->expert < y->expert ? -1 : 1;
+    if (x->flat != y->flat) return x->flat < y->flat ? -1 : 1;
+    return 0;
+}
+
+/* Reorder token rows by expert ([DS-AutoEP] runtime step 3; [DeepEP-272]
+ * dispatch on one device).  Assignments are sorted by the key (expert, flat
+ * index f = t*K + k) with the C library sort; the i-th assignment of expert e
+ * in that order lands on row offsets[e] + i.
+ *
+ *   x_perm[row(f)] = x[t]          flat_to_row[f] = row(f)
+ *   row_to_flat[row(f)] = f        all other rows: row_to_flat = -1
+ *   pad rows [offsets[e] + c_e, offsets[e+1]) are zero when zero_pad != 0;
+ *   rows [offsets[E], N_cap) keep their contents.
+ *
+ * Rows at or past N_cap are not written (ORC_CAPACITY). */
+int oracle_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
+                   const int32_t* offsets, int zero_pad, int64_t N_cap, uint16_t* x_perm,
+                   int32_t* row_to_flat, int32_t* flat_to_row) {
+    int status = 0;
+    int64_t A = (int64_t)T * K;
+    orc_assign* list = (orc_assign*)malloc(sizeof(orc_assign) * (size_t)(A > 0 ? A : 1));
+    int64_t n = 0;
+    for (int64_t f = 0; f < A; ++f) {
+        flat_to_row[f] = -1;
+        int64_t e = topk_idx[f];
+        if (e < 0 || e >= E) {
+            status |= ORC_EXPERT_OOR;
+            continue;
+        }
+        list[n].expert = (int32_t)e;
+        list[n].flat = (int32_t)f;
+        ++n;
+    }
+    qsort(list, (size_t)n, sizeof(orc_assign), orc_cmp_assign);
+
+    for (int64_t row = 0; row < N_cap; ++row) row_to_flat[row] = -1;
+    if ((int64_t)offsets[E] > N_cap) status |= ORC_CAPACITY;
+
+    int64_t i = 0;
+    while (i < n) {
+        int32_t e = list[i].expert;
+        int64_t j = i;
+        while (j < n && list[j].expert == e) {
+            int64_t row = (int64_t)offsets[e] + (j - i);
+            int32_t f = list[j].flat;
+            if (row < N_cap) {
+                int64_t t = f / K;
+                memcpy(x_perm + row * H, x + t * H, sizeof(uint16_t) * (size_t)H);
+                row_to_flat[row] = f;
+                flat_to_row[f] = (int32_t)row;
+            } else {
+                status |= ORC_CAPACITY;
+            }
+            ++j;
+        }
+        i = j;
+    }
+    if (zero_pad) {
+        for (int64_t row = 0; row < (int64_t)offsets[E] && row < N_cap; ++row)
+            if (row_to_flat[row] < 0) memset(x_perm + row * H, 0, sizeof(uint16_t) * (size_t)H);
+    }
+    free(list);
+    return status;
+}
+
+/* The definition of the row written for assignment f, counted by brute force
+ * in O(A^2): row(f) = offsets[e] + #{f' < f : topk_idx[f'] = e}.  Used only to
+ * pin oracle_permute on small inputs. */
+void oracle_bruteforce_rows(const int64_t* topk_idx, int T, int K, int E, const int32_t* offsets,
+                            int32_t* rows) {
+    int64_t A = (int64_t)T * K;
+    for (int64_t f = 0; f < A; ++f) {
+        int64_t e = topk_idx[f];
+        if (e < 0 || e >= E) {
+            rows[f] = -1;
+            continue;
+        }
+        int32_t before = 0;
+        for (int64_t g = 0; g < f; ++g)
+            if (topk_idx[g] == e) ++before;
+        rows[f] = offsets[e] + before;
+    }
+}
+
+/* ------------------------------------------------------ stand-in expert --- */
+
+/* The seeded per-expert stand-in y = x * s_e that sits where the grouped
+ * expert MLP would: every real row of expert e becomes
+ * bf16_rn(fp32(x) * s_e) -- the product of a bf16 and an fp32 is exact in
+ * fp64, rounded once to fp32 and then once to bf16.  Pad rows of expert e
+ * are written as zero; rows past offsets[E] are untouched. */
+void oracle_expert_scale(const uint16_t* rows, const int32_t* offsets,
+                         const int32_t* tokens_per_expert, int E, int H, const float* scales,
+                         uint16_t* out) {
+    for (int e = 0; e < E; ++e) {
+        int64_t begin = offsets[e];
+        int64_t real_end = begin + tokens_per_expert[e];
+        int64_t end = offsets[e + 1];
+        double s = (double)scales[e];
+        for (int64_t row = begin; row < end; ++row)
+            for (int h = 0; h < H; ++h) {
+                int64_t idx = row * H + h;
+                if (row < real_end) {
+                    double p = (double)oracle_float_from_bf16(rows[idx]) * s;
+                    out[idx] = oracle_bf16_from_float((float)p);
+                } else {
+                    out[idx] = 0;
+                }
+            }
+    }
+}
+
+/* ------------------------------------------------------------- combine --- */
+
+/* fused_weighted_restore [DS-8847] (Change; Benchmark): for every token t,
+ *
+ *   out[t] = sum_{k=0}^{K-1} w[t,k] * rows[flat_to_row[t*K+k]]
+ *
+ * with weights in the router dtype (passed here widened to float, which is
+ * exact for fp32 and bf16), or all ones when w == NULL (dispatch backward is
+ * a combine, [DeepEP-272]).  out_ref receives the fp64 sum (products are
+ * exact in fp64).  out_seq, when not NULL, receives the FP32 reading: acc = 0,
+ * then acc = fmaf(w, y, acc) for k = 0..K-1 in order, then one RNE to bf16.
+ * A slot whose row lies outside [0, N_cap) contributes nothing and sets
+ * ORC_ROW_OOR. */
+int oracle_combine(const uint16_t* rows, int64_t N_cap, const int32_t* flat_to_row,
+                   const float* w, int T, int K, int H, double* out_ref, uint16_t* out_seq) {
+    int status = 0;
+    for (int t = 0; t < T; ++t) {
+        for (int h = 0; h < H; ++h) {
+            double sum = 0.0;
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                int64_t f = (int64_t)t * K + k;
+                int64_t row = flat_to_row[f];
+                if (row < 0 || row >= N_cap) {
+                    status |= ORC_ROW_OOR;
+                    continue;
+                }
+                float wk = w ? w[f] : 1.0f;
+                float y = oracle_float_from_bf16(rows[row * H + h]);
+                sum += (double)wk * (double)y;
+                acc = fmaf(wk, y, acc);
+            }
+            out_ref[(int64_t)t * H + h] = sum;
+            if (out_seq) out_seq[(int64_t)t * H + h] = oracle_bf16_from_float(acc);
+        }
+    }
+    return status;
+}
+
+/* Coverage validation [DS-8847] (Change: "raises a clear RuntimeError if the
+ * gathered rows do not cover every (token, slot)"): every flat index f in
+ * [0, A) must be held by exactly one row.  Checked as the two maps being
+ * mutual inverses: row_to_flat[flat_to_row[f]] == f for every f, and
+ * flat_to_row[row_to_flat[r]] == r for every row r with row_to_flat[r] >= 0.
+ * Returns ORC_COVERAGE when either fails. */
+int oracle_check_coverage(const int32_t* row_to_flat, const int32_t* flat_to_row, int64_t N_cap,
+                          int64_t A) {
+    for (int64_t f = 0; f < A; ++f) {
+        int64_t row = flat_to_row[f];
+        if (row < 0 || row >= N_cap) return ORC_COVERAGE;
+        if (row_to_flat[row] != f) return ORC_COVERAGE;
+    }
+    for (int64_t row = 0; row < N_cap; ++row) {
+        int64_t f = row_to_flat[row];
+        if (f < 0) continue;
+        if (f >= A) return ORC_COVERAGE;
+        if (flat_to_row[f] != row) return ORC_COVERAGE;
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------- combine backward --- */
+
+/* The backward of fused_weighted_restore [DS-8847] (Tests: "row and score
+ * gradients"; Benchmark: score gradient in FP32).  With g = dL/d out:
+ *
+ *   grad_rows[flat_to_row[f]] = bf16_rn(fp32(w[f] * g[t]))
+ *   grad_w[f] = sum_h g[t,h] * rows[flat_to_row[f], h]       (fp64 sum)
+ *
+ * grad_w may be NULL.  When zero_pad != 0, every row below offsets[E] whose
+ * row_to_flat is negative (a pad row) is written as zero; rows at or past
+ * offsets[E] are untouched. */
+int oracle_combine_backward(const uint16_t* g, const uint16_t* rows, int64_t N_cap,
+                            const int32_t* row_to_flat, const int32_t* flat_to_row,
+                            const float* w, int T, int K, int H, const int32_t* offsets, int E,
+                            int zero_pad, uint16_t* grad_rows, double* grad_w) {
+    int status = 0;
+    for (int t = 0; t < T; ++t)
+        for (int k = 0; k < K; ++k) {
+            int64_t f = (int64_t)t * K + k;
+            int64_t row = flat_to_row[f];
+            if (row < 0 || row >= N_cap) {
+                status |= ORC_ROW_OOR;
+                if (grad_w) grad_w[f] = 0.0;
+                continue;
+            }
+            double wk = (double)w[f];
+            double dot = 0.0;
+            for (int h = 0; h < H; ++h) {
+                double gv = (double)oracle_float_from_bf16(g[(int64_t)t * H + h]);
+                double yv = (double)oracle_float_from_bf16(rows[row * H + h]);
+                grad_rows[row * H + h] = oracle_bf16_from_float((float)(wk * gv));
+                dot += gv * yv;
+            }
+            if (grad_w) grad_w[f] = dot;
+        }
+    if (zero_pad) {
+        for (int64_t row = 0; row < (int64_t)offsets[E] && row < N_cap; ++row)
+            if (row_to_flat[row] < 0) memset(grad_rows + row * H, 0, sizeof(uint16_t) * (size_t)H);
+    }
+    return status;
+}

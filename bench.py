@@ -1,0 +1,508 @@
+"""Benchmark: one step = the whole MoE dispatch/combine path, forward and
+backward, on synthetic seeded inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qwen3|dsv3|dsv3_skew|mixtral|tiny]
+
+Step (eight kernels, all through the C ABI of libmoe_dispatch.so):
+  layout (2 kernels) -> permute -> stand-in experts -> weighted combine
+  -> combine backward -> stand-in backward -> unit-weight combine.
+
+Default workload: Qwen3-MoE-shaped fwd+bwd (T=16384 tokens, H=2048, E=128 in
+8 logical ranks, top_k=8, fp32 router weights, mild skew, align 16): the one
+configuration that runs every step of the path, backward included.
+
+Prints ONE JSON line (rank 0).  ``value`` = tokens/s over all ranks (device
+time, CUDA events, max over ranks, L2 flushed by a 256 MiB write between
+steps), ``e2e`` = the same through pinned host buffers with the host<->device
+copies inside the timed region, ``roofline`` = the dominant kernel's
+algorithmic bytes per launch / its mean event-timed duration against the
+measured HBM copy bandwidth, ``cpu_baseline`` = the CPU oracle on a bounded
+sample of the same workload (rank 0, N=1).  With --impl reference the CPU
+oracle itself is timed as the reference arm.  N>1 runs independent replicas
+(the path has no exchange step on one device): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+KERNEL_SOURCES = {
+    "layout": "layout.cu", "permute": "permute.cu", "expert_scale": "expert_scale.cu",
+    "expert_scale_bwd": "expert_scale.cu", "combine": "combine.cu", "combine_backward": "combine.cu",
+    "dispatch_backward": "combine.cu",
+}
+
+
+# ------------------------------------------------------------------ setup ---
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(ws, backend="nccl"):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=180))
+        return dist
+    return None
+
+
+def max_over_ranks(dist, value: float, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(dist, tokens_per_rank: int, steps: int, total_ms: float, device):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    ws = dist.get_world_size() if dist is not None else 1
+    slowest = max_over_ranks(dist, total_ms, device)
+    return tokens_per_rank * ws * steps / (slowest / 1e3), slowest
+
+
+def barrier(dist, device):
+    if dist is not None:
+        dist.barrier(device_ids=[device.index] if device.type == "cuda" else None)
+
+
+# ------------------------------------------------------ algorithmic bytes ---
+
+def algorithmic_bytes(T, H, K, E, R, N_cap, N_pad):
+    """Bytes each launch must move (read + write) -- what the method needs,
+    not what the kernel happens to do.  P = pad rows = N_pad - A."""
+    A = T * K
+    P = N_pad - A
+    row = 2 * H
+    return {
+        "layout": 8 * A + T * R,
+        "permute": T * row + A * row + P * row + 8 * A + 4 * A + 4 * N_cap,
+        "expert_scale": A * row + N_pad * row,
+        "combine": A * row + T * row + 4 * A + 4 * A,
+        "combine_backward": T * row + A * row + A * row + P * row + 12 * A + 4 * N_pad,
+        "expert_scale_bwd": A * row + N_pad * row,
+        "dispatch_backward": A * row + T * row + 4 * A,
+    }
+
+
+# ----------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        ids = [v.strip() for v in vis.split(",")] if vis else []
+        self.gpu = ids[gpu_index] if gpu_index < len(ids) and ids[gpu_index] else str(gpu_index)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        try:
+            rows = [ln.split(",") for ln in open(self.path).read().strip().splitlines() if ln]
+            os.unlink(self.path)
+        except Exception:
+            return None
+        sm, mx, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1])); mx.append(float(r[2])); power.append(float(r[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------- ours ---
+
+class Path:
+    """Preallocated buffers and the eight launches of one step."""
+
+    def __init__(self, inp, cfg, device):
+        from combine_moe_dispatch_03_b200 import api
+        self.api = api
+        self.cfg = cfg
+        self.dev = device
+        T, H, E, K, R = cfg.T, cfg.H, cfg.E, cfg.K, cfg.R
+        self.x = inp["x"].to(device)
+        self.topk = inp["topk_idx"].to(device)
+        self.w = inp["weights"].to(device)
+        self.s = inp["scales"].to(device)
+        self.g = inp["grad_out"].to(device)
+        self.N = api.worst_case_rows(T, K, E, cfg.align)
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.status = api.new_status(device)
+        self.lay = api.alloc_layout(T, K, E, R, cfg.align, device)
+        self.xp = torch.zeros(self.N, H, **bf)
+        self.r2f = torch.empty(self.N, dtype=torch.int32, device=device)
+        self.f2r = torch.empty(T, K, dtype=torch.int32, device=device)
+        self.y = torch.zeros(self.N, H, **bf)
+        self.out = torch.empty(T, H, **bf)
+        self.grad_rows = torch.zeros(self.N, H, **bf)
+        self.grad_w = torch.empty(T, K, dtype=torch.float32, device=device)
+        self.grad_xp = torch.zeros(self.N, H, **bf)
+        self.grad_x = torch.empty(T, H, **bf)
+
+    names = ["layout", "permute", "expert_scale", "combine", "combine_backward", "expert_scale_bwd",
+             "dispatch_backward"]
+    kernels_per_step = 8   # layout is two kernels
+
+    def step(self, events=None):
+        api, c = self.api, self.cfg
+        st = self.status
+        ev = (lambda i: events[i].record()) if events is not None else (lambda i: None)
+        ev(0)
+        api.dispatch_layout(self.topk, c.E, c.R, c.align, status=st, out=self.lay)
+        ev(1)
+        api.permute(self.x, self.topk, self.lay, capacity=self.N, status=st,
+                    out=(self.xp, self.r2f, self.f2r))
+        ev(2)
+        api.expert_scale(self.xp, self.lay, self.s, status=st, out=self.y)
+        ev(3)
+        api.combine_weighted(self.y, self.f2r, self.w, status=st, out=self.out)
+        ev(4)
+        api.combine_backward(self.g, self.y, self.r2f, self.f2r, self.w, self.lay, status=st,
+                             out=(self.grad_rows, self.grad_w))
+        ev(5)
+        api.expert_scale(self.grad_rows, self.lay, self.s, status=st, out=self.grad_xp)
+        ev(6)
+        api.combine_weighted(self.grad_xp, self.f2r, None, status=st, out=self.grad_x)
+        ev(7)
+
+
+def kernel_source_sha(name: str) -> str:
+    p = os.path.join(ROOT, "combine_moe_dispatch_03_b200", "csrc", KERNEL_SOURCES[name])
+    h = hashlib.sha256()
+    for f in (p, os.path.join(ROOT, "combine_moe_dispatch_03_b200", "csrc", "common.cuh")):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(name: str, cfg_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the kernel source as it is now; else None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        d = json.load(open(p))
+        e = d[cfg_name][name]
+        if e.get("source_sha") == kernel_source_sha(name):
+            return e["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def run_ours(args, cfg, inp, dist, rank, ws, device):
+    from combine_moe_dispatch_03_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    if dist is not None:
+        dist.barrier()
+    _b.build()
+    path = Path(inp, cfg, device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.fill_(1)
+        path.step()
+    torch.cuda.synchronize(device)
+    path.api.check_status(path.status)
+
+    nk = len(Path.names) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk)] for _ in range(args.steps)]
+    sampler = ClockSampler(device.index)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    time.sleep(0.3)
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        path.step(evs[i])
+    torch.cuda.synchronize(device)
+    t_wall = time.perf_counter() - t_wall
+    clocks = sampler.stop()
+    barrier(dist, device)
+    path.api.check_status(path.status)
+
+    per_kernel = {n: [] for n in Path.names}
+    step_ms = []
+    for e in evs:
+        for j, n in enumerate(Path.names):
+            per_kernel[n].append(e[j].elapsed_time(e[j + 1]))
+        step_ms.append(e[0].elapsed_time(e[-1]))
+    total_ms = sum(step_ms)
+    value, total_ms_max = aggregate_throughput(dist, cfg.T, args.steps, total_ms, device)
+    ms_per_step = total_ms_max / args.steps
+
+    N_pad = int(path.lay.expert_offsets[-1].item())
+    nbytes = algorithmic_bytes(cfg.T, cfg.H, cfg.K, cfg.E, cfg.R, path.N, N_pad)
+    step_bytes = sum(nbytes.values())
+    mean_k = {n: statistics.fmean(v) for n, v in per_kernel.items()}
+    share = {n: sum(v) / total_ms for n, v in per_kernel.items()}
+    dom = max(per_kernel, key=lambda n: sum(per_kernel[n]))
+    peak, peak_kind = measured_peak()
+    achieved = nbytes[dom] / (mean_k[dom] / 1e3) / 1e9
+    hbm_gbs = step_bytes / (ms_per_step / 1e3) / 1e9
+
+    # ---- end to end: pinned host inputs -> device -> step -> host results ----
+    e2e = run_e2e(args, path, inp, dist, device, flush)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": cfg.description, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K,
+            "R": cfg.R, "align": cfg.align, "N_cap": path.N, "N_pad": N_pad,
+            "router_dtype": "fp32", "global_batch": cfg.T * ws, "parallelism": "replicas",
+            "l2": "flushed: 256 MiB device write between timed steps (outside the events)",
+            "step": "layout, permute, stand-in experts, combine, combine backward, "
+                    "stand-in backward, dispatch backward (unit-weight combine)",
+        },
+        "hbm": {"achieved_gbs": hbm_gbs, "bytes_per_step": step_bytes, "peak_gbs": peak,
+                "frac": hbm_gbs / peak, "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": ncu_traffic(dom, cfg.name),
+                     "bytes_per_launch": nbytes[dom], "mean_ms": mean_k[dom],
+                     "peak_kind": peak_kind},
+        "kernels": {n: {"mean_ms": mean_k[n], "share": share[n],
+                        "gbs": nbytes[n] / (mean_k[n] / 1e3) / 1e9} for n in Path.names},
+        "e2e": e2e,
+        "gpu_launches": Path.kernels_per_step * args.steps,
+        "clocks": clocks,
+        "wall_s_timed_region": t_wall,
+    }
+    return result
+
+
+def run_e2e(args, path, inp, dist, device, flush):
+    """Same metric through pinned host buffers: every step copies its inputs
+    host->device and its results (out, grad_x, grad_w) device->host."""
+    steps = max(3, min(args.steps, 50))
+    host_in = {k: inp[k].pin_memory() for k in ("x", "topk_idx", "weights", "scales", "grad_out")}
+    host_out = {"out": torch.empty_like(path.out, device="cpu").pin_memory(),
+                "grad_x": torch.empty_like(path.grad_x, device="cpu").pin_memory(),
+                "grad_w": torch.empty_like(path.grad_w, device="cpu").pin_memory()}
+    dev_in = {"x": path.x, "topk_idx": path.topk, "weights": path.w, "scales": path.s,
+              "grad_out": path.g}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def one(evpair=None):
+        if evpair:
+            evpair[0].record()
+        for k, t in host_in.items():
+            dev_in[k].copy_(t, non_blocking=True)
+        path.step()
+        host_out["out"].copy_(path.out, non_blocking=True)
+        host_out["grad_x"].copy_(path.grad_x, non_blocking=True)
+        host_out["grad_w"].copy_(path.grad_w, non_blocking=True)
+        if evpair:
+            evpair[1].record()
+
+    for _ in range(3):
+        flush.fill_(2)
+        one()
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    barrier(dist, device)
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        one(evs[i])
+    torch.cuda.synchronize(device)
+    total = sum(a.elapsed_time(b) for a, b in evs)
+    value, total = aggregate_throughput(dist, path.cfg.T, steps, total, device)
+    return {"value": value, "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": total / steps}
+
+
+# ------------------------------------------------------ CPU oracle timing ---
+
+def oracle_step(orc, sample):
+    """One pass of the whole path through the CPU oracle (single thread)."""
+    s = sample
+    lay = orc.layout(s["topk"], s["E"], s["R"], s["align"])
+    pm = orc.permute(s["x"], s["topk"], s["E"], lay["expert_offsets"], s["N"])
+    y = orc.expert_scale(pm["x_perm"], lay["expert_offsets"], lay["tokens_per_expert"], s["s"])
+    orc.combine(y, pm["flat_to_row"], s["w"], seq=False)
+    bw = orc.combine_backward(s["g"], y, pm["row_to_flat"], pm["flat_to_row"], s["w"],
+                              lay["expert_offsets"])
+    gxp = orc.expert_scale(bw["grad_rows"], lay["expert_offsets"], lay["tokens_per_expert"], s["s"])
+    orc.combine(gxp, pm["flat_to_row"], None, seq=False)
+
+
+def oracle_sample(cfg, inp, tokens):
+    from combine_moe_dispatch_03_b200.inputs import bf16_bits
+    T = min(tokens, cfg.T)
+    T -= T % cfg.R
+    return dict(x=bf16_bits(inp["x"][:T]), topk=inp["topk_idx"][:T].numpy(),
+                w=inp["weights"][:T].numpy(), s=inp["scales"].numpy(),
+                g=bf16_bits(inp["grad_out"][:T]), E=cfg.E, R=cfg.R, align=cfg.align, T=T,
+                N=T * cfg.K + cfg.E * (cfg.align - 1))
+
+
+def time_oracle(cfg, inp, min_s=10.0, max_s=30.0, tokens=1024):
+    import oracle as orc
+    orc.build()
+    sample = oracle_sample(cfg, inp, tokens)
+    oracle_step(orc, sample)   # warm (page-in)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(orc, sample)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_s or (el >= max_s * 0.5 and n >= 1):
+            break
+    return {"value": sample["T"] * n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {sample['T']} tokens of the workload (same H, E, K, R, align), "
+                      f"whole fwd+bwd path, {n} passes in {el:.1f} s, single-threaded C"}
+
+
+def run_reference(args, cfg, inp, rank, ws):
+    """The CPU oracle timed as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle as orc
+    orc.build()
+    # size the per-step sample so that warm-up + timed steps take ~2 minutes
+    probe = oracle_sample(cfg, inp, 256)
+    t0 = time.perf_counter()
+    oracle_step(orc, probe)
+    per_token = (time.perf_counter() - t0) / probe["T"]
+    budget = 120.0 / (args.steps + args.warmup)
+    tokens = int(max(cfg.R, min(cfg.T, budget / max(per_token, 1e-9))))
+    sample = oracle_sample(cfg, inp, tokens)
+    for _ in range(max(args.warmup, 0)):
+        oracle_step(orc, sample)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(orc, sample)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = sample["T"] * args.steps / total
+    desc = (f"first {sample['T']} tokens of the workload per step (same H, E, K, R, align), "
+            "whole fwd+bwd path, single-threaded C oracle")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.description, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K,
+                   "R": cfg.R, "align": cfg.align, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------- main ---
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen3")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    sys.path.insert(0, ROOT)
+    from combine_moe_dispatch_03_b200.inputs import CONFIGS, make_inputs
+    cfg = CONFIGS[args.workload]
+    ws, rank, local = dist_env()
+
+    if args.impl == "reference":
+        inp = make_inputs(cfg, with_grad=True)
+        res = run_reference(args, cfg, inp, rank, ws)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(ws)
+    try:
+        inp = make_inputs(cfg, seed=cfg.seed + rank, with_grad=True)
+        res = run_ours(args, cfg, inp, dist, rank, ws, device)
+        if rank == 0:
+            if ws == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = time_oracle(cfg, inp)
+            else:
+                res["cpu_baseline"] = None
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,219 @@
+"""Python entry points over the C ABI -- argument marshalling only.
+
+Every function takes CUDA tensors, allocates its outputs with torch (device
+memory from the caching allocator, no host synchronisation), and enqueues the
+library's kernels on the current torch stream.  Device-side errors accumulate
+in an int32 ``status`` tensor; ``check_status`` reads it (one sync) and raises
+a RuntimeError naming the bits, the way the coverage check of
+fused_weighted_restore raises (DeepSpeed PR "AutoEP: support
+combine_impl=fused_weighted_sum with AutoEP+AutoTP folding", Change).
+
+The names follow the C ABI: dispatch_layout / permute / expert_scale /
+combine_weighted / combine_backward.  A ``Layout`` plus the two row maps play
+the part of DeepEP's dispatch ``handle`` (DeepEP issue "Does Deepep's
+Dispatch/Combine Support Autograd Like PyTorch's all_to_all?").
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+from . import _lib
+from ._lib import DTYPE_BF16, DTYPE_F32, check_rc, lib
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device):
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int | None = None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def _weight_dtype(w: torch.Tensor) -> int:
+    if w.dtype == torch.float32:
+        return DTYPE_F32
+    if w.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    raise TypeError(f"weights must be float32 or bfloat16 (router dtype), got {w.dtype}")
+
+
+def new_status(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def check_status(status: torch.Tensor) -> None:
+    """Synchronise once on ``status`` and raise if any kernel flagged bad data."""
+    bits = int(status.item())
+    if bits:
+        raise RuntimeError("MoE dispatch/combine device check failed: "
+                           + "; ".join(_lib.decode_status(bits)) + f" (status bits {bits:#x})")
+
+
+def worst_case_rows(T: int, K: int, E: int, align: int) -> int:
+    n = lib().moe_worst_case_rows(T, K, E, align)
+    if n < 0:
+        raise ValueError("invalid sizes")
+    return int(n)
+
+
+def workspace_bytes(T: int, K: int, E: int, R: int) -> int:
+    n = lib().moe_layout_workspace_bytes(T, K, E, R)
+    if n == 0:
+        raise ValueError("invalid sizes for the layout workspace")
+    return int(n)
+
+
+@dataclasses.dataclass
+class Layout:
+    """Outputs of moe_dispatch_layout (all device tensors)."""
+    tokens_per_expert: torch.Tensor   # [E] int32
+    counts: torch.Tensor              # [R, R, E/R] int32
+    splits: torch.Tensor              # [R, R] int32
+    tokens_per_rank: torch.Tensor     # [R, R] int32
+    is_token_in_rank: torch.Tensor    # [T, R] uint8
+    expert_offsets: torch.Tensor      # [E+1] int32
+    workspace: torch.Tensor           # opaque, uint8
+    T: int
+    K: int
+    E: int
+    R: int
+    align: int
+
+
+def alloc_layout(T: int, K: int, E: int, R: int, align: int, device) -> Layout:
+    i32 = dict(dtype=torch.int32, device=device)
+    return Layout(
+        tokens_per_expert=torch.empty(E, **i32),
+        counts=torch.empty(R, R, E // R, **i32),
+        splits=torch.empty(R, R, **i32),
+        tokens_per_rank=torch.empty(R, R, **i32),
+        is_token_in_rank=torch.empty(T, R, dtype=torch.uint8, device=device),
+        expert_offsets=torch.empty(E + 1, **i32),
+        workspace=torch.empty(workspace_bytes(T, K, E, R), dtype=torch.uint8, device=device),
+        T=T, K=K, E=E, R=R, align=align)
+
+
+def dispatch_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int = 1,
+                    align: int = 1, status: torch.Tensor | None = None,
+                    out: Layout | None = None) -> Layout:
+    _require(topk_idx, "topk_idx", torch.int64, 2)
+    T, K = topk_idx.shape
+    dev = topk_idx.device
+    lay = out if out is not None else alloc_layout(T, K, num_experts, num_ranks, align, dev)
+    st = status if status is not None else new_status(dev)
+    rc = lib().moe_dispatch_layout(
+        _ptr(topk_idx), T, K, num_experts, num_ranks, align, _ptr(lay.tokens_per_expert),
+        _ptr(lay.counts), _ptr(lay.splits), _ptr(lay.tokens_per_rank), _ptr(lay.is_token_in_rank),
+        _ptr(lay.expert_offsets), _ptr(lay.workspace), _ptr(st), _stream(dev))
+    check_rc(rc, "moe_dispatch_layout")
+    return lay
+
+
+def permute(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout, capacity: int | None = None,
+            zero_pad: bool = True, status: torch.Tensor | None = None,
+            out: tuple | None = None):
+    """Returns (x_perm [N_cap,H] bf16, row_to_flat [N_cap] int32, flat_to_row [T,K] int32)."""
+    _require(x, "x", torch.bfloat16, 2)
+    _require(topk_idx, "topk_idx", torch.int64, 2)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    dev = x.device
+    N_cap = capacity if capacity is not None else worst_case_rows(T, K, layout.E, layout.align)
+    if out is None:
+        x_perm = torch.empty(N_cap, H, dtype=torch.bfloat16, device=dev)
+        r2f = torch.empty(N_cap, dtype=torch.int32, device=dev)
+        f2r = torch.empty(T, K, dtype=torch.int32, device=dev)
+    else:
+        x_perm, r2f, f2r = out
+    st = status if status is not None else new_status(dev)
+    rc = lib().moe_permute(_ptr(x), _ptr(topk_idx), T, K, layout.E, H, _ptr(layout.expert_offsets),
+                           _ptr(layout.workspace), int(bool(zero_pad)), N_cap, _ptr(x_perm),
+                           _ptr(r2f), _ptr(f2r), _ptr(st), _stream(dev))
+    check_rc(rc, "moe_permute")
+    return x_perm, r2f, f2r
+
+
+def expert_scale(rows: torch.Tensor, layout: Layout, scales: torch.Tensor,
+                 status: torch.Tensor | None = None, out: torch.Tensor | None = None):
+    """Stand-in expert: y = bf16_rn(rows * s_e) on real rows, 0 on pad rows."""
+    _require(rows, "rows", torch.bfloat16, 2)
+    _require(scales, "scales", torch.float32, 1)
+    N_cap, H = rows.shape
+    y = out if out is not None else torch.empty_like(rows)
+    st = status if status is not None else new_status(rows.device)
+    rc = lib().moe_expert_scale(_ptr(rows), N_cap, _ptr(layout.expert_offsets),
+                                _ptr(layout.tokens_per_expert), layout.E, H, _ptr(scales), _ptr(y),
+                                _ptr(st), _stream(rows.device))
+    check_rc(rc, "moe_expert_scale")
+    return y
+
+
+def combine_weighted(rows: torch.Tensor, flat_to_row: torch.Tensor,
+                     weights: torch.Tensor | None = None, row_to_flat: torch.Tensor | None = None,
+                     validate: bool = False, status: torch.Tensor | None = None,
+                     out: torch.Tensor | None = None):
+    """fused_weighted_restore; weights=None is the unit-weight combine
+    (the backward of dispatch)."""
+    _require(rows, "rows", torch.bfloat16, 2)
+    _require(flat_to_row, "flat_to_row", torch.int32, 2)
+    N_cap, H = rows.shape
+    T, K = flat_to_row.shape
+    wd = DTYPE_F32
+    if weights is not None:
+        wd = _weight_dtype(weights)
+        _require(weights, "weights", weights.dtype, 2)
+        if tuple(weights.shape) != (T, K):
+            raise ValueError("weights must be [T, K]")
+    if validate:
+        if row_to_flat is None:
+            raise ValueError("validate=True needs row_to_flat")
+        _require(row_to_flat, "row_to_flat", torch.int32, 1)
+    o = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=rows.device)
+    st = status if status is not None else new_status(rows.device)
+    rc = lib().moe_combine_weighted(_ptr(rows), N_cap, _ptr(row_to_flat), _ptr(flat_to_row),
+                                    _ptr(weights), wd, T, K, H, int(bool(validate)), _ptr(o),
+                                    _ptr(st), _stream(rows.device))
+    check_rc(rc, "moe_combine_weighted")
+    return o
+
+
+def combine_backward(grad_out: torch.Tensor, rows: torch.Tensor, row_to_flat: torch.Tensor,
+                     flat_to_row: torch.Tensor, weights: torch.Tensor, layout: Layout,
+                     zero_pad: bool = True, want_grad_weights: bool = True,
+                     status: torch.Tensor | None = None, out: tuple | None = None):
+    """Returns (grad_rows [N_cap,H] bf16, grad_weights [T,K] router dtype or None)."""
+    _require(grad_out, "grad_out", torch.bfloat16, 2)
+    _require(rows, "rows", torch.bfloat16, 2)
+    _require(flat_to_row, "flat_to_row", torch.int32, 2)
+    _require(row_to_flat, "row_to_flat", torch.int32, 1)
+    wd = _weight_dtype(weights)
+    _require(weights, "weights", weights.dtype, 2)
+    N_cap, H = rows.shape
+    T, K = flat_to_row.shape
+    if out is None:
+        grad_rows = torch.empty_like(rows)
+        grad_w = torch.empty(T, K, dtype=weights.dtype, device=rows.device) if want_grad_weights else None
+    else:
+        grad_rows, grad_w = out
+    st = status if status is not None else new_status(rows.device)
+    rc = lib().moe_combine_backward(_ptr(grad_out), _ptr(rows), N_cap, _ptr(row_to_flat),
+                                    _ptr(flat_to_row), _ptr(weights), wd, T, K, H,
+                                    _ptr(layout.expert_offsets), layout.E, int(bool(zero_pad)),
+                                    _ptr(grad_rows), _ptr(grad_w), _ptr(st), _stream(rows.device))
+    check_rc(rc, "moe_combine_backward")
+    return grad_rows, grad_w

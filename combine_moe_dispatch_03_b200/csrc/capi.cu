@@ -1,0 +1,186 @@
+// capi.cu -- the extern "C" entry points of libmoe_dispatch.so: argument
+// checks on the host, then kernel launches on the caller's stream.  No call
+// allocates, synchronises or reads device memory on the host.
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "internal.h"
+#include "moe_dispatch.h"
+
+namespace moe {
+
+// Per-device SM count (the only state kept between calls).
+int sm_count_current_device() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64) {
+        int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+}  // namespace moe
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Sizes shared by the calls; see the limits in moe_dispatch.h.
+bool sizes_ok(int T, int K, int E) {
+    if (T < 0 || K < 1 || K > MOE_MAX_K || E < 1 || E > MOE_MAX_E) return false;
+    if ((int64_t)T * K > INT32_MAX) return false;
+    return true;
+}
+
+bool hidden_ok(int H) { return H > 0 && (H % 8) == 0; }
+
+bool ncap_ok(int64_t N_cap, int T, int K) {
+    return N_cap >= (int64_t)T * K && N_cap <= INT32_MAX;
+}
+
+int finish(cudaError_t err) { return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_layout_workspace_bytes(int T, int K, int E, int R) {
+    if (!sizes_ok(T, K, E) || R < 1 || R > MOE_MAX_R || E % R || T % R) return 0;
+    const moe::Geometry g = moe::layout_geometry(T, K, R);
+    return moe::workspace_layout(E, R, g.n_tiles).total;
+}
+
+int64_t moe_worst_case_rows(int T, int K, int E, int align) {
+    if (!sizes_ok(T, K, E) || align < 1) return -1;
+    return (int64_t)T * K + (int64_t)E * (align - 1);
+}
+
+int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int align,
+                        int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                        int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
+                        int32_t* expert_offsets, void* workspace, int32_t* status,
+                        cudaStream_t stream) {
+    if (!sizes_ok(T, K, E) || R < 1 || R > MOE_MAX_R || E % R || T % R || align < 1)
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)T * K + (int64_t)E * (align - 1) > INT32_MAX) return MOE_ERR_INVALID_ARG;
+    if (!tokens_per_expert || !counts || !splits || !tokens_per_rank || !expert_offsets ||
+        !workspace || !status)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !is_token_in_rank)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, 8) || !aligned(workspace, 16) || !aligned(tokens_per_expert, 4) ||
+        !aligned(counts, 4) || !aligned(splits, 4) || !aligned(tokens_per_rank, 4) ||
+        !aligned(expert_offsets, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    return finish(moe::launch_layout(topk_idx, T, K, E, R, align, tokens_per_expert, counts,
+                                     splits, tokens_per_rank, is_token_in_rank, expert_offsets,
+                                     workspace, status, stream));
+}
+
+int moe_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
+                const int32_t* expert_offsets, const void* workspace, int zero_pad,
+                int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat, int32_t* flat_to_row,
+                int32_t* status, cudaStream_t stream) {
+    if (!sizes_ok(T, K, E) || !hidden_ok(H) || !ncap_ok(N_cap, T, K)) return MOE_ERR_INVALID_ARG;
+    if (!expert_offsets || !workspace || !status) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !topk_idx || !flat_to_row)) return MOE_ERR_INVALID_ARG;
+    if (N_cap > 0 && (!x_perm || !row_to_flat)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(topk_idx, 8) ||
+        !aligned(workspace, 16) || !aligned(expert_offsets, 4) || !aligned(row_to_flat, 4) ||
+        !aligned(flat_to_row, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    return finish(moe::launch_permute(x, topk_idx, T, K, E, H, expert_offsets, workspace,
+                                      zero_pad, N_cap, x_perm, row_to_flat, flat_to_row, status,
+                                      stream));
+}
+
+int moe_expert_scale(const uint16_t* rows, int64_t N_cap, const int32_t* expert_offsets,
+                     const int32_t* tokens_per_expert, int E, int H, const float* scales,
+                     uint16_t* out, int32_t* status, cudaStream_t stream) {
+    if (E < 1 || E > MOE_MAX_E || !hidden_ok(H) || N_cap < 0 || N_cap > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (!expert_offsets || !tokens_per_expert || !scales || !status) return MOE_ERR_INVALID_ARG;
+    if (N_cap > 0 && (!rows || !out)) return MOE_ERR_INVALID_ARG;
+    if (N_cap > 0 && rows == out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(rows, 16) || !aligned(out, 16) || !aligned(expert_offsets, 4) ||
+        !aligned(tokens_per_expert, 4) || !aligned(scales, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    return finish(moe::launch_expert_scale(rows, N_cap, expert_offsets, tokens_per_expert, E, H,
+                                           scales, out, status, stream));
+}
+
+int moe_combine_weighted(const uint16_t* rows, int64_t N_cap, const int32_t* row_to_flat,
+                         const int32_t* flat_to_row, const void* weights, int weight_dtype,
+                         int T, int K, int H, int validate, uint16_t* out, int32_t* status,
+                         cudaStream_t stream) {
+    if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || !hidden_ok(H) ||
+        N_cap < 0 || N_cap > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (weight_dtype != MOE_DTYPE_F32 && weight_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (!status) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!flat_to_row || !out)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && N_cap > 0 && !rows) return MOE_ERR_INVALID_ARG;
+    if (validate && N_cap > 0 && !row_to_flat) return MOE_ERR_INVALID_ARG;
+    const size_t wal = weight_dtype == MOE_DTYPE_F32 ? 4 : 2;
+    if (!aligned(rows, 16) || !aligned(out, 16) || !aligned(flat_to_row, 4) ||
+        !aligned(row_to_flat, 4) || !aligned(weights, wal) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0 && !validate) return MOE_OK;
+    return finish(moe::launch_combine(rows, N_cap, row_to_flat, flat_to_row, weights, weight_dtype,
+                                      T, K, H, validate, out, status, stream));
+}
+
+int moe_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t N_cap,
+                         const int32_t* row_to_flat, const int32_t* flat_to_row,
+                         const void* weights, int weight_dtype, int T, int K, int H,
+                         const int32_t* expert_offsets, int E, int zero_pad,
+                         uint16_t* grad_rows, void* grad_weights, int32_t* status,
+                         cudaStream_t stream) {
+    if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || !hidden_ok(H) ||
+        N_cap < 0 || N_cap > INT32_MAX || E < 1 || E > MOE_MAX_E)
+        return MOE_ERR_INVALID_ARG;
+    if (weight_dtype != MOE_DTYPE_F32 && weight_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (!status || !expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!grad_out || !flat_to_row || !weights)) return MOE_ERR_INVALID_ARG;
+    if (N_cap > 0 && (!rows || !grad_rows)) return MOE_ERR_INVALID_ARG;
+    if (zero_pad && N_cap > 0 && !row_to_flat) return MOE_ERR_INVALID_ARG;
+    const size_t wal = weight_dtype == MOE_DTYPE_F32 ? 4 : 2;
+    if (!aligned(grad_out, 16) || !aligned(rows, 16) || !aligned(grad_rows, 16) ||
+        !aligned(flat_to_row, 4) || !aligned(row_to_flat, 4) || !aligned(weights, wal) ||
+        !aligned(grad_weights, wal) || !aligned(expert_offsets, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0 && !zero_pad) return MOE_OK;
+    return finish(moe::launch_combine_backward(grad_out, rows, N_cap, row_to_flat, flat_to_row,
+                                               weights, weight_dtype, T, K, H, expert_offsets, E,
+                                               zero_pad, grad_rows, grad_weights, status, stream));
+}
+
+const char* moe_strerror(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument (null pointer, size outside the limits, or misaligned buffer)";
+        case MOE_ERR_CUDA: return "CUDA launch or runtime error";
+        default: return "unknown return code";
+    }
+}
+
+const char* moe_status_bit_name(int bit) {
+    switch (bit) {
+        case MOE_ST_EXPERT_OOR: return "topk_idx entry outside [0, E)";
+        case MOE_ST_CAPACITY: return "padded rows exceed the row capacity N_cap";
+        case MOE_ST_ROW_OOR: return "flat_to_row entry outside [0, N_cap)";
+        case MOE_ST_COVERAGE: return "row maps do not cover every (token, slot) exactly once";
+        case MOE_ST_LAYOUT_MISMATCH: return "layout workspace was built for other sizes";
+        default: return "unknown status bit";
+    }
+}
+
+const char* moe_version(void) { return "moe_dispatch 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,98 @@
+// internal.h -- launchers behind the C ABI and the layout workspace format.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Layout workspace: [header | tile_base (E x n_tiles) | tile_tpr (n_tiles x R)
+// | expert_count (E)], each part 256-byte aligned.  Tiles are runs of at most
+// TT consecutive tokens that never straddle two source ranks' token blocks, so
+// per-rank sums are sums over whole tiles.  tile_base[e][j] first holds the
+// number of expert-e assignments in tile j, then (after the scan) the number
+// in all earlier tiles: the stable base of tile j inside expert e's group.
+struct LayoutHeader {
+    int64_t off_tile_base;     // byte offsets of the parts (so a reader needs no R)
+    int64_t off_tile_tpr;
+    int64_t off_expert_count;
+    int32_t magic;
+    int32_t T, K, E, R;
+    int32_t TT;        // tokens per tile
+    int32_t tpb;       // tiles per source block
+    int32_t n_tiles;   // R * tpb
+    uint32_t done;     // arrival counter of the scan kernel (self-resetting)
+};
+static_assert(sizeof(LayoutHeader) == 64, "header is 64 bytes");
+
+constexpr int32_t kLayoutMagic = 0x4d6f4531;  // "MoE1"
+constexpr int kMaxTileAssign = 512;          // TT * K <= this
+
+struct Geometry {
+    int TT, tpb, n_tiles;
+};
+
+// Tile geometry: about 4 tiles per SM of a 148-SM B200 for the large configs,
+// at most kMaxTileAssign assignments per tile.  A pure function of the sizes,
+// so the workspace size is known before any device is touched.
+inline Geometry layout_geometry(int T, int K, int R) {
+    const int Tb = R > 0 ? T / R : 0;
+    int tt = (T + 591) / 592;
+    int cap = kMaxTileAssign / K;
+    if (tt > cap) tt = cap;
+    if (tt < 1) tt = 1;
+    if (Tb > 0 && tt > Tb) tt = Tb;
+    Geometry g;
+    g.TT = tt;
+    g.tpb = Tb > 0 ? (Tb + tt - 1) / tt : 0;
+    g.n_tiles = R * g.tpb;
+    return g;
+}
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct WsLayout {
+    size_t tile_base, tile_tpr, expert_count, total;
+};
+
+inline WsLayout workspace_layout(int E, int R, int n_tiles) {
+    WsLayout w;
+    w.tile_base = align256(sizeof(LayoutHeader));
+    w.tile_tpr = w.tile_base + align256(sizeof(int32_t) * (size_t)E * (size_t)n_tiles);
+    w.expert_count = w.tile_tpr + align256(sizeof(int32_t) * (size_t)n_tiles * (size_t)R);
+    w.total = w.expert_count + align256(sizeof(int32_t) * (size_t)E);
+    return w;
+}
+
+int sm_count_current_device();
+
+cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int align,
+                          int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                          int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
+                          int32_t* expert_offsets, void* workspace, int32_t* status,
+                          cudaStream_t stream);
+
+cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
+                           const int32_t* expert_offsets, const void* workspace, int zero_pad,
+                           int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat,
+                           int32_t* flat_to_row, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_expert_scale(const uint16_t* rows, int64_t N_cap, const int32_t* expert_offsets,
+                                const int32_t* tokens_per_expert, int E, int H,
+                                const float* scales, uint16_t* out, int32_t* status,
+                                cudaStream_t stream);
+
+cudaError_t launch_combine(const uint16_t* rows, int64_t N_cap, const int32_t* row_to_flat,
+                           const int32_t* flat_to_row, const void* weights, int weight_dtype,
+                           int T, int K, int H, int validate, uint16_t* out, int32_t* status,
+                           cudaStream_t stream);
+
+cudaError_t launch_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t N_cap,
+                                    const int32_t* row_to_flat, const int32_t* flat_to_row,
+                                    const void* weights, int weight_dtype, int T, int K, int H,
+                                    const int32_t* expert_offsets, int E, int zero_pad,
+                                    uint16_t* grad_rows, void* grad_weights, int32_t* status,
+                                    cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,235 @@
+/*
+ * moe_dispatch.h -- C ABI of libmoe_dispatch.so: Mixture-of-Experts token
+ * dispatch and combine on one NVIDIA B200 (sm_100a).
+ *
+ * The path, in call order (forward, then backward):
+ *
+ *   moe_dispatch_layout   routing layout from topk_idx           (integer)
+ *   moe_permute           token rows -> expert-grouped buffer    (byte copy)
+ *   moe_expert_scale      stand-in expert y = x * s_e            (fp32, one rounding)
+ *   moe_combine_weighted  weighted top-k gather-sum -> tokens    (fp32 accumulate)
+ *   moe_combine_backward  row gradients + routing-weight grads   (fp32 / fp64)
+ *   moe_combine_weighted  with weights = NULL: dispatch backward (fp32 accumulate)
+ *
+ * Sources (titles of the pages that define the operations):
+ *   [DeepEP-272] DeepEP issue "Does Deepep's Dispatch/Combine Support Autograd
+ *                Like PyTorch's all_to_all?": get_dispatch_layout and its
+ *                outputs; the backward of dispatch is a combine and the
+ *                backward of combine is a dispatch; the handle; a worst-case
+ *                size instead of a CPU wait (num_worst_tokens).
+ *   [DS-8847]    DeepSpeed PR "AutoEP: support combine_impl=fused_weighted_sum
+ *                with AutoEP+AutoTP folding", sections Problem, Change, Tests,
+ *                Benchmark: fused_weighted_restore, flat index token*top_k +
+ *                slot, router-dtype weights as [tokens, top_k], FP32
+ *                accumulation, the coverage error, row and score gradients.
+ *   [DS-AutoEP]  DeepSpeed AutoEP base PR, sections Attribution and Design:
+ *                reorder tokens by expert, token-group alignment / padding for
+ *                grouped GEMM, restore the original order.
+ *   [DS-8190]    DeepSpeed PR "Derive AutoEP rank splits from the per-expert
+ *                count exchange", sections Redundancy and Fix: the count
+ *                matrix [ep_size, E_local], input_splits and
+ *                received_counts.sum(dim=1) == output_splits.
+ *   [XTuner-2056] XTuner PR "Integrate MoonEP dispatcher for FSDP
+ *                expert-parallel training", Design and review: no host
+ *                synchronisation on the hot path (histc, not bincount).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every data pointer is caller-owned DEVICE memory of the current device.
+ *    The library allocates nothing and never synchronises with the host;
+ *    every call only enqueues kernels on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) and returns.  Results are defined once the
+ *    stream reaches them.  The only state kept between calls is a per-device
+ *    cache of the SM count.
+ *  - Notation: T tokens, H hidden size (bf16 elements per row), E experts,
+ *    K = top_k, R logical ranks, El = E/R, align = group alignment,
+ *    A = T*K assignments, flat index f = t*K + k (token t, slot k),
+ *    N_cap = rows of the caller's expert-grouped buffers.
+ *    Logical rank s owns tokens [s*T/R, (s+1)*T/R) as a source and experts
+ *    [r*El, (r+1)*El) as a destination.  All arrays are row-major, densely
+ *    packed.  bf16 values are passed as their uint16 bit patterns.
+ *  - Return value: a HOST-detected error, MOE_OK (0) or a negative
+ *    MOE_ERR_* code; on error nothing is enqueued.
+ *  - `status` is one DEVICE int32 the caller zeroes before the first call;
+ *    kernels OR MOE_ST_* bits into it when they meet bad data on the device.
+ *    Outputs of a call that set a bit are undefined, but no kernel ever
+ *    writes outside the buffers described here.  Read it after the stream
+ *    has reached it (one synchronisation, when the caller chooses).
+ *  - Limits: 1 <= K <= MOE_MAX_K, 1 <= E <= MOE_MAX_E, 1 <= R <= MOE_MAX_R,
+ *    E % R == 0, T % R == 0, T >= 0, H > 0 and H % 8 == 0 (rows are whole
+ *    16-byte vectors), A and N_cap < 2^31.  Row buffers must be 16-byte
+ *    aligned, int64 arrays 8-byte, int32/float arrays 4-byte aligned.
+ */
+#ifndef MOE_DISPATCH_H
+#define MOE_DISPATCH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host return codes. */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1) /* a check listed under the call failed      */
+#define MOE_ERR_CUDA (-2)        /* a CUDA runtime call or launch failed      */
+
+/* Device status bits (OR-ed into *status). */
+#define MOE_ST_EXPERT_OOR 1       /* a topk_idx entry outside [0, E) (e.g. -1)  */
+#define MOE_ST_CAPACITY 2         /* padded rows expert_offsets[E] > N_cap      */
+#define MOE_ST_ROW_OOR 4          /* a flat_to_row entry outside [0, N_cap)     */
+#define MOE_ST_COVERAGE 8         /* row maps do not cover each (token, slot) once */
+#define MOE_ST_LAYOUT_MISMATCH 16 /* workspace was built for another (T, K, E)  */
+
+/* Routing-weight ("router") dtypes. */
+#define MOE_DTYPE_F32 0
+#define MOE_DTYPE_BF16 1
+
+#define MOE_MAX_K 32
+#define MOE_MAX_E 1024
+#define MOE_MAX_R 64
+
+/* Bytes of the opaque layout workspace for (T, K, E, R).  The workspace is
+ * written by moe_dispatch_layout and read by moe_permute (it plays the part of
+ * the dispatch handle of [DeepEP-272]: per-tile expert bases and per-expert
+ * counts).  Needs no initialisation.  Returns 0 for invalid sizes. */
+size_t moe_layout_workspace_bytes(int T, int K, int E, int R);
+
+/* A capacity that every routing fits: A + E*(align-1) rows (each expert
+ * rounds its count up to a multiple of align).  Sizing the grouped buffers
+ * with it removes the host wait for the actual count ([DeepEP-272],
+ * num_worst_tokens).  Returns -1 for invalid sizes. */
+int64_t moe_worst_case_rows(int T, int K, int E, int align);
+
+/* Routing layout ([DeepEP-272] get_dispatch_layout; [DS-8190] count matrix;
+ * [DS-AutoEP] group alignment).  Computed on the device only, with no host
+ * synchronisation ([XTuner-2056]).
+ *
+ * In:  topk_idx [T,K] int64, entries in [0, E).
+ * Out: tokens_per_expert [E] int32    c_e = #{f : topk_idx[f] = e}
+ *      counts  [R,R,El] int32         counts[s][r][el] = assignments from
+ *                                     source rank s to expert r*El+el (row s
+ *                                     is rank s's count matrix [ep_size,
+ *                                     E_local]; counts[:, r, :] is the
+ *                                     received_counts of rank r)
+ *      splits  [R,R] int32            splits[s][r] = sum_el counts[s][r][el]
+ *                                     (row s = input_splits of rank s,
+ *                                     column r = output_splits of rank r)
+ *      tokens_per_rank [R,R] int32    distinct tokens of block s with some
+ *                                     slot on rank r (num_tokens_per_rank)
+ *      is_token_in_rank [T,R] uint8   1 iff some slot of t routes to rank r
+ *      expert_offsets [E+1] int32     0, then running sum of
+ *                                     ceil(c_e/align)*align (an empty expert
+ *                                     takes no rows)
+ *      workspace                      moe_layout_workspace_bytes(T,K,E,R)
+ *                                     bytes, 16-byte aligned
+ * Status: MOE_ST_EXPERT_OOR (that assignment is left out of every count).
+ * Errors: MOE_ERR_INVALID_ARG for a null pointer, sizes outside the limits,
+ *         align < 1, misalignment. */
+int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int align,
+                        int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                        int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
+                        int32_t* expert_offsets, void* workspace, int32_t* status,
+                        cudaStream_t stream);
+
+/* Dispatch on one device ([DeepEP-272] dispatch; [DS-AutoEP] step 3,
+ * "reorder tokens by expert assignment").  Assignment f = (t, k) with
+ * e = topk_idx[f] is written to
+ *
+ *   row(f) = expert_offsets[e] + #{f' < f : topk_idx[f'] = e}
+ *
+ * (stable order: expert, then token, then slot):
+ *   x_perm[row(f)] = x[t],  flat_to_row[f] = row(f),  row_to_flat[row(f)] = f.
+ * Pad rows [off[e] + c_e, off[e+1]) get row_to_flat = -1 and, when zero_pad
+ * is non-zero, zero contents.  Rows [off[E], N_cap) get row_to_flat = -1 and
+ * keep their contents.
+ *
+ * In:  x [T,H] bf16; topk_idx [T,K] int64; expert_offsets and workspace from
+ *      moe_dispatch_layout with the same (topk_idx, T, K, E).
+ * Out: x_perm [N_cap,H] bf16, row_to_flat [N_cap] int32, flat_to_row [T,K]
+ *      int32 (-1 for an assignment that was not placed).
+ * Status: MOE_ST_CAPACITY (rows >= N_cap are not written),
+ *         MOE_ST_EXPERT_OOR, MOE_ST_LAYOUT_MISMATCH (nothing written).
+ * Errors: MOE_ERR_INVALID_ARG as for the layout, or N_cap < A. */
+int moe_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
+                const int32_t* expert_offsets, const void* workspace, int zero_pad,
+                int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat, int32_t* flat_to_row,
+                int32_t* status, cudaStream_t stream);
+
+/* Stand-in expert between dispatch and combine: for each expert e, its real
+ * rows [off[e], off[e] + c_e) become bf16_rn(fp32(row) * scales[e]) (the
+ * product rounded to fp32, then once to bf16); its pad rows become zero;
+ * rows >= off[E] are untouched.  In the backward pass the same call maps row
+ * gradients to input-row gradients (d(x*s)/dx = s).  It stands where the
+ * grouped expert MLP of [DS-AutoEP] (Design, step 5) runs.
+ *
+ * In:  rows [N_cap,H] bf16; expert_offsets [E+1]; tokens_per_expert [E];
+ *      scales [E] fp32.   Out: out [N_cap,H] bf16 (may not alias rows).
+ * Status: MOE_ST_CAPACITY if off[E] > N_cap (nothing past N_cap is touched). */
+int moe_expert_scale(const uint16_t* rows, int64_t N_cap, const int32_t* expert_offsets,
+                     const int32_t* tokens_per_expert, int E, int H, const float* scales,
+                     uint16_t* out, int32_t* status, cudaStream_t stream);
+
+/* fused_weighted_restore ([DS-8847] Change; [DeepEP-272] combine):
+ *
+ *   acc = 0;  for k = 0..K-1:  acc = fmaf(w[t,k], rows[flat_to_row[t*K+k]], acc)
+ *   out[t] = bf16_rn(acc)
+ *
+ * per element, FP32, fixed slot order, one rounding.  weights [T,K] are in the
+ * router dtype (weight_dtype = MOE_DTYPE_F32 or MOE_DTYPE_BF16, widened
+ * exactly); weights = NULL means unit weights, which is the backward of
+ * dispatch ([DeepEP-272]: "the backward process of MoE dispatch is actually a
+ * combine").  A slot whose row is outside [0, N_cap) contributes nothing and
+ * sets MOE_ST_ROW_OOR.
+ *
+ * validate != 0 adds the coverage check of [DS-8847] ("raises a clear
+ * RuntimeError if the gathered rows do not cover every (token, slot)"):
+ * row_to_flat[flat_to_row[f]] == f for every f, and
+ * flat_to_row[row_to_flat[r]] == r for every row with row_to_flat[r] >= 0;
+ * a failure sets MOE_ST_COVERAGE.  row_to_flat may be NULL when validate == 0.
+ *
+ * In:  rows [N_cap,H] bf16, maps from moe_permute.   Out: out [T,H] bf16. */
+int moe_combine_weighted(const uint16_t* rows, int64_t N_cap, const int32_t* row_to_flat,
+                         const int32_t* flat_to_row, const void* weights, int weight_dtype,
+                         int T, int K, int H, int validate, uint16_t* out, int32_t* status,
+                         cudaStream_t stream);
+
+/* Backward of fused_weighted_restore ([DS-8847] Tests: row and score
+ * gradients; Benchmark: score gradient in FP32; [DeepEP-272]: the backward
+ * of combine is a dispatch).  With g = grad_out [T,H]:
+ *
+ *   grad_rows[flat_to_row[f]] = bf16_rn(fp32(w[f] * g[t]))
+ *   grad_weights[f] = sum_h g[t,h] * rows[flat_to_row[f], h]
+ *
+ * grad_weights: bf16 x bf16 products are exact in fp32 and are summed in
+ * fp64, then rounded once to the router dtype; it may be NULL.  When zero_pad
+ * is non-zero, every row below expert_offsets[E] whose row_to_flat is
+ * negative (a pad row) is written as zero; rows >= off[E] are untouched.
+ * row_to_flat may be NULL when zero_pad == 0.
+ *
+ * In:  grad_out [T,H] bf16; rows [N_cap,H] bf16 (the forward's combine input);
+ *      maps; weights [T,K] (router dtype, not NULL); expert_offsets [E+1].
+ * Out: grad_rows [N_cap,H] bf16; grad_weights [T,K] router dtype.
+ * Status: MOE_ST_ROW_OOR (that slot is skipped and its weight gradient is 0). */
+int moe_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t N_cap,
+                         const int32_t* row_to_flat, const int32_t* flat_to_row,
+                         const void* weights, int weight_dtype, int T, int K, int H,
+                         const int32_t* expert_offsets, int E, int zero_pad,
+                         uint16_t* grad_rows, void* grad_weights, int32_t* status,
+                         cudaStream_t stream);
+
+/* Static text for a return code (MOE_OK / MOE_ERR_*) or for ONE status bit. */
+const char* moe_strerror(int code);
+const char* moe_status_bit_name(int bit);
+
+/* Library version string. */
+const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DISPATCH_H */

@@ -1,0 +1,149 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, element by
+element, on the seeded workloads and on edge cases.
+
+Bar: bit-exact for layout, offsets, row maps, permuted rows, stand-in rows and
+row gradients; |gpu - oracle| <= 2^-7 |oracle| + 1e-6 for the combine output,
+the weight gradient and the dispatch-backward output (the FP32 slot-order
+value is additionally expected bit-exact).
+"""
+import numpy as np
+import pytest
+import torch
+
+from _pipeline import SENTINEL, compare, run_gpu, run_oracle
+from combine_moe_dispatch_03_b200.inputs import CONFIGS, capacity_rows, custom_inputs, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from combine_moe_dispatch_03_b200 import build
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _check(inp, E, R, align, N_cap=None, **kw):
+    T, K = inp["topk_idx"].shape
+    if N_cap is None:
+        N_cap = capacity_rows(T, K, E, align)
+    gpu = run_gpu(inp, E, R, align, N_cap, **kw)
+    ref = run_oracle(inp, E, R, align, N_cap, zero_pad=kw.get("zero_pad", True),
+                     weights=kw.get("weights"), backward=kw.get("backward", True))
+    compare(gpu, ref, backward=kw.get("backward", True),
+            bf16_weights=kw.get("weights") is not None and kw["weights"].dtype == torch.bfloat16)
+    return gpu, ref
+
+
+# ------------------------------------------------------- seeded workloads ---
+
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "dsv3_skew", "qwen3"])
+def test_config_full_size(name):
+    """Every output of every call at the workload's full size, forward and
+    backward, with the capacity and launch configuration the bench uses."""
+    cfg = CONFIGS[name]
+    inp = make_inputs(name, with_grad=True)
+    _check(inp, cfg.E, cfg.R, cfg.align)
+
+
+def test_tiny_twice_deterministic():
+    cfg = CONFIGS["tiny"]
+    inp = make_inputs("tiny", with_grad=True)
+    N = capacity_rows(cfg.T, cfg.K, cfg.E, cfg.align)
+    a = run_gpu(inp, cfg.E, cfg.R, cfg.align, N)
+    b = run_gpu(inp, cfg.E, cfg.R, cfg.align, N)
+    for k in ("x_perm", "flat_to_row", "out", "grad_rows", "grad_w", "grad_x"):
+        np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+# ------------------------------------------------------------ edge cases ---
+
+@pytest.mark.parametrize("T,H,E,K,R,align", [
+    (1, 8, 1, 1, 1, 1),          # smallest everything
+    (3, 16, 3, 2, 1, 2),         # hand-example sizes
+    (1000, 136, 7, 3, 1, 4),     # ragged T, H not a multiple of 32 vectors, odd K
+    (997, 264, 13, 5, 1, 8),     # prime T, K=5
+    (640, 64, 16, 6, 8, 16),     # K=6, 8 logical ranks
+    (512, 72, 32, 7, 4, 3),      # K=7, align 3
+    (300, 40, 40, 9, 4, 1),      # K=9 (generic paths)
+    (64, 32, 64, 32, 2, 2),      # K=32 (maximum)
+    (256, 16, 1024, 4, 64, 1),   # E=1024 and R=64 (maxima)
+    (130, 8192, 8, 2, 2, 16),    # wide rows
+])
+def test_edge_shapes(T, H, E, K, R, align):
+    inp = custom_inputs(T, H, E, K, seed=T * 7 + K)
+    _check(inp, E, R, align)
+
+
+def test_empty_input():
+    inp = custom_inputs(0, 64, 4, 2, seed=1)
+    gpu, ref = _check(inp, 4, 2, 8, N_cap=16)
+    assert np.all(gpu["row_to_flat"] == -1)
+
+
+def test_all_tokens_on_one_expert():
+    T, K, E = 776, 4, 16
+    topk = torch.zeros(T, K, dtype=torch.int64)
+    topk[:, 1] = 5                         # a repeated expert within a token
+    topk[:, 3] = 15
+    inp = custom_inputs(T, 128, E, K, seed=5, topk_idx=topk)
+    _check(inp, E, 4, 16)
+    topk[:] = 2                            # every slot of every token on one expert
+    inp = custom_inputs(T, 128, E, K, seed=6, topk_idx=topk)
+    _check(inp, E, 1, 128)
+
+
+def test_repeated_experts_and_skew():
+    g = torch.Generator().manual_seed(3)
+    T, K, E = 2048, 8, 64
+    topk = torch.randint(0, 4, (T, K), generator=g)        # heavy repeats on 4 experts
+    topk[::3] = torch.randint(0, E, (len(range(0, T, 3)), K), generator=g)
+    inp = custom_inputs(T, 256, E, K, seed=9, topk_idx=topk)
+    _check(inp, E, 8, 16)
+
+
+def test_no_zero_pad_leaves_pad_rows():
+    cfg = CONFIGS["tiny"]
+    inp = make_inputs("tiny", with_grad=True)
+    gpu, ref = _check(inp, cfg.E, cfg.R, cfg.align, zero_pad=False)
+    r2f = gpu["row_to_flat"]
+    N_pad = gpu["expert_offsets"][-1]
+    pads = np.nonzero(r2f[:N_pad] < 0)[0]
+    assert len(pads) > 0
+    assert np.all(gpu["x_perm"][pads] == SENTINEL)
+
+
+def test_bf16_router_weights():
+    cfg = CONFIGS["tiny"]
+    inp = make_inputs("tiny", with_grad=True)
+    _check(inp, cfg.E, cfg.R, cfg.align, weights=inp["weights"].to(torch.bfloat16))
+
+
+def test_logical_ranks_do_not_change_rows():
+    """R only regroups the counts: rows, maps and outputs are identical for
+    R = 1 and R = 8 on the same routing (partitioned == unpartitioned)."""
+    cfg = CONFIGS["qwen3"]
+    inp = make_inputs("qwen3", T=2048, with_grad=True)
+    N = capacity_rows(2048, cfg.K, cfg.E, cfg.align)
+    a = run_gpu(inp, cfg.E, 1, cfg.align, N)
+    b = run_gpu(inp, cfg.E, 8, cfg.align, N)
+    for k in ("x_perm", "row_to_flat", "flat_to_row", "y", "out", "grad_rows", "grad_w", "grad_x",
+              "expert_offsets", "tokens_per_expert"):
+        np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+def test_combine_token_chunks_concatenate():
+    """Combining two halves of the tokens gives the same bytes as all at once."""
+    from combine_moe_dispatch_03_b200 import api
+    cfg = CONFIGS["tiny"]
+    inp = make_inputs("tiny", T=512)
+    dev = torch.device("cuda:0")
+    lay = api.dispatch_layout(inp["topk_idx"].to(dev), cfg.E, cfg.R, cfg.align)
+    xp, r2f, f2r = api.permute(inp["x"].to(dev), inp["topk_idx"].to(dev), lay)
+    w = inp["weights"].to(dev)
+    full = api.combine_weighted(xp, f2r, w)
+    h = 256
+    a = api.combine_weighted(xp, f2r[:h].contiguous(), w[:h].contiguous())
+    b = api.combine_weighted(xp, f2r[h:].contiguous(), w[h:].contiguous())
+    assert torch.equal(full.view(torch.int16), torch.cat([a, b]).view(torch.int16))

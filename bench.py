@@ -307,7 +307,7 @@ def run_ours(args, cfg, inp, dist, rank, ws, device):
     hbm_gbs = step_bytes / (ms_per_step / 1e3) / 1e9
 
     # ---- end to end: pinned host inputs -> device -> step -> host results ----
-    e2e = run_e2e(args, path, inp, dist, device, flush)
+    e2e = None if args.no_e2e else run_e2e(args, path, inp, dist, device, flush)
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
@@ -471,6 +471,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (profiling of smaller cases; must divide by R)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -478,6 +481,10 @@ def main():
     sys.path.insert(0, ROOT)
     from combine_moe_dispatch_03_b200.inputs import CONFIGS, make_inputs
     cfg = CONFIGS[args.workload]
+    if args.tokens is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, T=args.tokens,
+                                  description=cfg.description + f" (T overridden to {args.tokens})")
     ws, rank, local = dist_env()
 
     if args.impl == "reference":

@@ -89,7 +89,9 @@ combine_kernel(const uint16_t* __restrict__ rows, int64_t N_cap, const int32_t* 
                 }
             }
         } else {
-            for (int c = lane; c < n16; c += 32 * U) {
+            // Warp-uniform trip count: the shuffles inside need all 32 lanes.
+            for (int c0 = 0; c0 < n16; c0 += 32 * U) {
+                const int c = c0 + lane;
                 float acc[U][8];
 #pragma unroll
                 for (int u = 0; u < U; ++u)

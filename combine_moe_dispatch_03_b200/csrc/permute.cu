@@ -94,7 +94,10 @@ permute_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ topk,
         for (int q = warp; q < ntok; q += kWarps) {
             const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(t0 + q) * H);
             const int myrow = (lane < K) ? rowi[q * K + lane] : -1;
-            for (int c = lane; c < n16; c += 32 * U) {
+            // Warp-uniform trip count (the shuffles below need all 32 lanes);
+            // accesses past the row end are predicated off.
+            for (int c0 = 0; c0 < n16; c0 += 32 * U) {
+                const int c = c0 + lane;
                 uint4 v[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u)

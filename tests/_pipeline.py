@@ -99,8 +99,10 @@ def run_oracle(inp: dict, E: int, R: int, align: int, N_cap: int, *, zero_pad=Tr
     y = orc.expert_scale(pm["x_perm"], lay["expert_offsets"], lay["tokens_per_expert"], s,
                          out_init=init)
     cb = orc.combine(y, pm["flat_to_row"], w32)
-    res = dict(lay, **pm, y=y, out_ref=cb["ref"], out_seq=cb["seq"], status=lay["status"] |
-               pm["status"] | cb["status"])
+    res = dict(lay)
+    res.update(pm)
+    res.update(y=y, out_ref=cb["ref"], out_seq=cb["seq"],
+               status=lay["status"] | pm["status"] | cb["status"])
     if backward:
         g = bf16_bits(inp["grad_out"])
         bw = orc.combine_backward(g, y, pm["row_to_flat"], pm["flat_to_row"], w32,

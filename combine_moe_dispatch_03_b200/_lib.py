@@ -15,6 +15,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_disp
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = -1
 MOE_ERR_CUDA = -2
+MOE_ERR_SCRATCH = -3
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 ST_EXPERT_OOR = 1
 ST_CAPACITY = 2
@@ -38,6 +40,7 @@ SIGNATURES = {
     "moe_layout_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "moe_worst_case_rows": (ctypes.c_int64, [_I, _I, _I, _I]),
     "moe_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_dispatch_layout_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _L, _P, _P, _P, _P, _P]),
     "moe_expert_scale": (_I, [_P, _L, _P, _P, _I, _I, _P, _P, _P, _P]),
     "moe_combine_weighted": (_I, [_P, _L, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),

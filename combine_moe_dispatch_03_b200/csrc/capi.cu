@@ -166,6 +166,7 @@ const char* moe_strerror(int code) {
         case MOE_OK: return "ok";
         case MOE_ERR_INVALID_ARG: return "invalid argument (null pointer, size outside the limits, or misaligned buffer)";
         case MOE_ERR_CUDA: return "CUDA launch or runtime error";
+        case MOE_ERR_SCRATCH: return "sizes exceed the static scratch of moe_dispatch_layout_noalloc (MOE_NOALLOC_SCRATCH_BYTES)";
         default: return "unknown return code";
     }
 }

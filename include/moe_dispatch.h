@@ -76,6 +76,8 @@ extern "C" {
 #define MOE_OK 0
 #define MOE_ERR_INVALID_ARG (-1) /* a check listed under the call failed      */
 #define MOE_ERR_CUDA (-2)        /* a CUDA runtime call or launch failed      */
+#define MOE_ERR_SCRATCH (-3)     /* sizes need more than the static scratch of
+                                    moe_dispatch_layout_noalloc              */
 
 /* Device status bits (OR-ed into *status). */
 #define MOE_ST_EXPERT_OOR 1       /* a topk_idx entry outside [0, E) (e.g. -1)  */
@@ -87,6 +89,9 @@ extern "C" {
 /* Routing-weight ("router") dtypes. */
 #define MOE_DTYPE_F32 0
 #define MOE_DTYPE_BF16 1
+
+/* Bytes of the static device scratch behind moe_dispatch_layout_noalloc. */
+#define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
 
 #define MOE_MAX_K 32
 #define MOE_MAX_E 1024
@@ -134,6 +139,35 @@ int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int
                         int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
                         int32_t* expert_offsets, void* workspace, int32_t* status,
                         cudaStream_t stream);
+
+/* moe_dispatch_layout for callers that cannot allocate device memory.  The
+ * pages have no counterpart of this call; it exists for callers such as a
+ * plugin running inside a server or framework that owns the whole device
+ * memory pool and only hands over the tensors it passes, or a path where
+ * cudaMalloc/cudaFree must not run because they can synchronise the device.
+ *
+ * Same arguments, outputs, status bits and errors as moe_dispatch_layout,
+ * minus `workspace`: the layout's scratch lives in one file-scope device
+ * array of MOE_NOALLOC_SCRATCH_BYTES (4 MiB) that every GPU which loads the
+ * library holds until the process exits.  The caller still passes all inputs
+ * and outputs.  The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *  - Sizes whose workspace (moe_layout_workspace_bytes(T, K, E, R)) exceeds
+ *    MOE_NOALLOC_SCRATCH_BYTES are rejected with MOE_ERR_SCRATCH and nothing
+ *    is enqueued.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture on the device.
+ *  - Every call shares the one array, which keeps the last call's contents
+ *    (the kernels rewrite every word they read, so nothing needs clearing).
+ *    Calls that overlap on the GPU -- on different streams, or from threads
+ *    whose streams are not ordered -- race on it and give undefined results.
+ *  - The permute cannot use this scratch; a caller that also permutes uses
+ *    moe_dispatch_layout with its own workspace. */
+int moe_dispatch_layout_noalloc(const int64_t* topk_idx, int T, int K, int E, int R, int align,
+                                int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                                int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
+                                int32_t* expert_offsets, int32_t* status, cudaStream_t stream);
 
 /* Dispatch on one device ([DeepEP-272] dispatch; [DS-AutoEP] step 3,
  * "reorder tokens by expert assignment").  Assignment f = (t, k) with

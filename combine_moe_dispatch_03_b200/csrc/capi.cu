@@ -54,7 +54,7 @@ extern "C" {
 size_t moe_layout_workspace_bytes(int T, int K, int E, int R) {
     if (!sizes_ok(T, K, E) || R < 1 || R > MOE_MAX_R || E % R || T % R) return 0;
     const moe::Geometry g = moe::layout_geometry(T, K, R);
-    return moe::workspace_layout(E, R, g.n_tiles).total;
+    return moe::workspace_layout(E, R, g.n_tiles, (int64_t)T * K).total;
 }
 
 int64_t moe_worst_case_rows(int T, int K, int E, int align) {

@@ -16,25 +16,26 @@
 //     grad_rows[row(t,k)] = bf16_rn(fp32(w[t,k] * g[t]))
 //     grad_w[t,k] = sum_h g[t,h] * y[row(t,k), h]   (exact fp32 products, fp64 sum)
 //
-// One warp per token, grid-stride.  Lane k < K fetches slot k's row index and
-// weight once; the row indices are then broadcast to registers, so for every
-// 16-byte column chunk the warp issues the K gathers back to back (K*U
-// vectors in flight per lane) before the fixed-order FMA chain.  Reads are
-// coalesced 512-byte row segments; the output row is written once.
+// The gathers are what cost: K scattered rows per token.  DRAM serves them
+// best as long contiguous runs, so for K <= 8 the kernels are "slot-major":
+// a warp walks the slots in order and fetches a contiguous 1-4 KB chunk of
+// each slot's row, keeping D chunks in flight (a ring in registers), instead
+// of fetching a 512-byte sliver of all K rows at once.  For K > 8 a generic
+// warp-per-token kernel serves any K.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
-// ------------------------------------------------------------- forward ---
-
-template <int KT, int U, bool VALIDATE>
+// ------------------------------------------------- forward, any K ---
+// One warp per token; for each column chunk of 32 x U vectors the slots are
+// visited in order (any K up to MOE_MAX_K).
+template <int U, bool VALIDATE>
 __global__ void __launch_bounds__(kBlock)
 combine_kernel(const uint16_t* __restrict__ rows, int64_t N_cap, const int32_t* __restrict__ r2f,
                const int32_t* __restrict__ f2r, const void* __restrict__ w, int wdtype, int T,
                int K, int H, uint16_t* __restrict__ out, int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int Kn = KT > 0 ? KT : K;
     const int n16 = H >> 3;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     int bad = 0;
@@ -42,8 +43,8 @@ combine_kernel(const uint16_t* __restrict__ rows, int64_t N_cap, const int32_t* 
     for (int t = blockIdx.x * kWarps + warp; t < T; t += gridDim.x * kWarps) {
         int myrow = -1;
         float myw = 0.f;
-        if (lane < Kn) {
-            const int64_t f = (int64_t)t * Kn + lane;
+        if (lane < K) {
+            const int64_t f = (int64_t)t * K + lane;
             int r = f2r[f];
             if (r < 0 || (int64_t)r >= N_cap) {
                 bad |= MOE_ST_ROW_OOR;
@@ -55,76 +56,41 @@ combine_kernel(const uint16_t* __restrict__ rows, int64_t N_cap, const int32_t* 
             myrow = r;
         }
         uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * H);
-        if constexpr (KT > 0) {
-            int rk[KT];
-            float wk[KT];
+        // Warp-uniform trip count: the shuffles inside need all 32 lanes.
+        for (int c0 = 0; c0 < n16; c0 += 32 * U) {
+            const int c = c0 + lane;
+            float acc[U][8];
 #pragma unroll
-            for (int k = 0; k < KT; ++k) {
-                rk[k] = __shfl_sync(kFull, myrow, k);
-                wk[k] = __shfl_sync(kFull, myw, k);
-            }
-            for (int c = lane; c < n16; c += 32 * U) {
-                uint4 v[KT][U];
+            for (int u = 0; u < U; ++u)
 #pragma unroll
-                for (int k = 0; k < KT; ++k) {
-                    const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[k] < 0 ? 0 : rk[k]) * H);
+                for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+            for (int k = 0; k < K; ++k) {
+                const int r = __shfl_sync(kFull, myrow, k);
+                const float wv = __shfl_sync(kFull, myw, k);
+                if (r < 0) continue;
+                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)r * H);
+                uint4 v[U];
 #pragma unroll
-                    for (int u = 0; u < U; ++u)
-                        v[k][u] = (rk[k] >= 0 && c + 32 * u < n16) ? ld_stream(src + c + 32 * u) : zero;
-                }
+                for (int u = 0; u < U; ++u)
+                    v[u] = (c + 32 * u < n16) ? ld_stream(src + c + 32 * u) : zero;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    if (c + 32 * u >= n16) continue;
-                    float acc[8];
+                    float y[8];
+                    unpack8(v[u], y);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll
-                    for (int k = 0; k < KT; ++k) {
-                        float y[8];
-                        unpack8(v[k][u], y);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(wk[k], y[i], acc[i]);
-                    }
-                    st_vec(dst + c + 32 * u, pack8(acc));
+                    for (int i = 0; i < 8; ++i) acc[u][i] = __fmaf_rn(wv, y[i], acc[u][i]);
                 }
             }
-        } else {
-            // Warp-uniform trip count: the shuffles inside need all 32 lanes.
-            for (int c0 = 0; c0 < n16; c0 += 32 * U) {
-                const int c = c0 + lane;
-                float acc[U][8];
 #pragma unroll
-                for (int u = 0; u < U; ++u)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-                for (int k = 0; k < Kn; ++k) {
-                    const int r = __shfl_sync(kFull, myrow, k);
-                    const float wv = __shfl_sync(kFull, myw, k);
-                    if (r < 0) continue;
-                    const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)r * H);
-                    uint4 v[U];
-#pragma unroll
-                    for (int u = 0; u < U; ++u)
-                        v[u] = (c + 32 * u < n16) ? ld_stream(src + c + 32 * u) : zero;
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        float y[8];
-                        unpack8(v[u], y);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) acc[u][i] = __fmaf_rn(wv, y[i], acc[u][i]);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < U; ++u)
-                    if (c + 32 * u < n16) st_vec(dst + c + 32 * u, pack8(acc[u]));
-            }
+            for (int u = 0; u < U; ++u)
+                if (c + 32 * u < n16) st_vec(dst + c + 32 * u, pack8(acc[u]));
         }
     }
 
     if (VALIDATE) {
         // Row side of the bijection: every row that claims a (token, slot)
         // must be the row that (token, slot) points to.
-        const int64_t A = (int64_t)T * Kn;
+        const int64_t A = (int64_t)T * K;
         const int64_t stride = (int64_t)gridDim.x * kBlock;
         for (int64_t row = (int64_t)blockIdx.x * kBlock + threadIdx.x; row < N_cap; row += stride) {
             const int32_t f = r2f[row];
@@ -135,9 +101,114 @@ combine_kernel(const uint16_t* __restrict__ rows, int64_t N_cap, const int32_t* 
     warp_status_or(status, bad);
 }
 
-// ------------------------------------------------------------ backward ---
+// ------------------------------------------------- forward, slot-major ---
+//
+// One warp per (token, column chunk) item; a chunk is 32 lanes x U 16-byte
+// vectors (2 KB for U = 4).  The warp walks the slots k = 0..K-1 in order
+// and, for each, loads that slot's row chunk -- a contiguous run, the access
+// pattern DRAM serves best -- keeping D row chunks in flight (a ring), and
+// applies acc = fmaf(w_k, y, acc) as each chunk lands.  Same arithmetic and
+// order as combine_kernel.
+#ifndef MOE_COMBINE_U
+#define MOE_COMBINE_U 2
+#endif
+#ifndef MOE_COMBINE_D
+#define MOE_COMBINE_D 4
+#endif
 
-template <int KT, int U>
+template <int KT, int U, int D, bool VALIDATE>
+__global__ void __launch_bounds__(kBlock)
+combine_slots_kernel(const uint16_t* __restrict__ rows, int64_t N_cap,
+                     const int32_t* __restrict__ r2f, const int32_t* __restrict__ f2r,
+                     const void* __restrict__ w, int wdtype, int T, int H,
+                     uint16_t* __restrict__ out, int32_t* __restrict__ status) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n16 = H >> 3;
+    const int chunks = (n16 + 32 * U - 1) / (32 * U);
+    const int64_t n_items = (int64_t)T * chunks;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    int bad = 0;
+
+    for (int64_t item = (int64_t)blockIdx.x * kWarps + warp; item < n_items;
+         item += (int64_t)gridDim.x * kWarps) {
+        const int64_t t = item / chunks;
+        const int c = (int)(item - t * chunks);
+        int myrow = -1;
+        float myw = 0.f;
+        if (lane < KT) {
+            const int64_t f = t * KT + lane;
+            int r = f2r[f];
+            if (r < 0 || (int64_t)r >= N_cap) {
+                if (c == 0) bad |= MOE_ST_ROW_OOR;
+                r = -1;
+            } else {
+                myw = w ? load_weight(w, wdtype, f) : 1.f;
+                if (VALIDATE && c == 0 && r2f[r] != (int32_t)f) bad |= MOE_ST_COVERAGE;
+            }
+            myrow = r;
+        }
+        int rk[KT];
+        float wk[KT];
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+            rk[k] = __shfl_sync(kFull, myrow, k);
+            wk[k] = __shfl_sync(kFull, myw, k);
+        }
+        const int v0 = c * 32 * U + lane;
+        uint4 ring[D][U];
+#pragma unroll
+        for (int k = 0; k < D && k < KT; ++k) {
+            const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[k] < 0 ? 0 : rk[k]) * H);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                ring[k][u] = (rk[k] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
+        }
+        float acc[U][8];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+            const int slot = k % D;
+            if (rk[k] >= 0) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    float y[8];
+                    unpack8(ring[slot][u], y);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[u][i] = __fmaf_rn(wk[k], y[i], acc[u][i]);
+                }
+            }
+            if (k + D < KT) {
+                const int kn = k + D;
+                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[kn] < 0 ? 0 : rk[kn]) * H);
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    ring[slot][u] = (rk[kn] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
+            }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * H);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (v0 + 32 * u < n16) st_vec(dst + v0 + 32 * u, pack8(acc[u]));
+    }
+
+    if (VALIDATE) {
+        const int64_t A = (int64_t)T * KT;
+        const int64_t stride = (int64_t)gridDim.x * kBlock;
+        for (int64_t row = (int64_t)blockIdx.x * kBlock + threadIdx.x; row < N_cap; row += stride) {
+            const int32_t f = r2f[row];
+            if (f < 0) continue;
+            if ((int64_t)f >= A || (int64_t)f2r[f] != row) bad |= MOE_ST_COVERAGE;
+        }
+    }
+    warp_status_or(status, bad);
+}
+
+// ------------------------------------------------ backward, any K ---
+// One warp per token, one slot at a time over the whole row (g is re-read
+// per slot from cache); the weight gradient is reduced per slot.
 __global__ void __launch_bounds__(kBlock)
 combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ rows,
                    int64_t N_cap, const int32_t* __restrict__ r2f,
@@ -165,104 +236,38 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
             myrow = r;
         }
         const uint4* gsrc = reinterpret_cast<const uint4*>(g + (size_t)t * H);
-        if constexpr (KT == 0) {
-            // Any K: one slot at a time over the whole row (g is re-read per
-            // slot from cache); the weight gradient is reduced per slot.
-            for (int k = 0; k < K; ++k) {
-                const int r = __shfl_sync(kFull, myrow, k);
-                const float wv = __shfl_sync(kFull, myw, k);
-                double dk = 0.0;
-                if (r >= 0) {
-                    const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)r * H);
-                    uint4* dst = reinterpret_cast<uint4*>(grad_rows + (size_t)r * H);
-                    for (int c = lane; c < n16; c += 32) {
-                        float gf[8], yf[8], o[8];
-                        unpack8(gsrc[c], gf);
-                        unpack8(ld_stream(src + c), yf);
-                        double part = 0.0;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            part += (double)__fmul_rn(gf[i], yf[i]);
-                            o[i] = __fmul_rn(wv, gf[i]);
-                        }
-                        dk += part;
-                        st_vec(dst + c, pack8(o));
-                    }
-                }
-#pragma unroll
-                for (int d = 16; d > 0; d >>= 1) dk += __shfl_xor_sync(kFull, dk, d);
-                if (grad_w && lane == 0) {
-                    const int64_t f = (int64_t)t * K + k;
-                    if (wdtype == MOE_DTYPE_F32) {
-                        static_cast<float*>(grad_w)[f] = __double2float_rn(dk);
-                    } else {
-                        __nv_bfloat16 b = __double2bfloat16(dk);
-                        static_cast<uint16_t*>(grad_w)[f] = *reinterpret_cast<uint16_t*>(&b);
-                    }
-                }
-            }
-            continue;
-        } else {
-        int rk[KT];
-        float wk[KT];
-        double dot[KT];
-#pragma unroll
-        for (int k = 0; k < KT; ++k) {
-            rk[k] = __shfl_sync(kFull, myrow, k);
-            wk[k] = __shfl_sync(kFull, myw, k);
-            dot[k] = 0.0;
-        }
-        for (int c = lane; c < n16; c += 32 * U) {
-            uint4 gv[U];
-            uint4 yv[KT][U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) gv[u] = (c + 32 * u < n16) ? ld_stream(gsrc + c + 32 * u) : zero;
-#pragma unroll
-            for (int k = 0; k < KT; ++k) {
-                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[k] < 0 ? 0 : rk[k]) * H);
-#pragma unroll
-                for (int u = 0; u < U; ++u)
-                    yv[k][u] = (rk[k] >= 0 && c + 32 * u < n16) ? ld_stream(src + c + 32 * u) : zero;
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                if (c + 32 * u >= n16) continue;
-                float gf[8];
-                unpack8(gv[u], gf);
-#pragma unroll
-                for (int k = 0; k < KT; ++k) {
-                    if (rk[k] < 0) continue;
-                    float yf[8], o[8];
-                    unpack8(yv[k][u], yf);
+        for (int k = 0; k < K; ++k) {
+            const int r = __shfl_sync(kFull, myrow, k);
+            const float wv = __shfl_sync(kFull, myw, k);
+            double dk = 0.0;
+            if (r >= 0) {
+                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)r * H);
+                uint4* dst = reinterpret_cast<uint4*>(grad_rows + (size_t)r * H);
+                for (int c = lane; c < n16; c += 32) {
+                    float gf[8], yf[8], o[8];
+                    unpack8(gsrc[c], gf);
+                    unpack8(ld_stream(src + c), yf);
                     double part = 0.0;
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         part += (double)__fmul_rn(gf[i], yf[i]);   // exact: bf16 x bf16
-                        o[i] = __fmul_rn(wk[k], gf[i]);
+                        o[i] = __fmul_rn(wv, gf[i]);
                     }
-                    dot[k] += part;
-                    uint4* dst = reinterpret_cast<uint4*>(grad_rows + (size_t)rk[k] * H);
-                    st_vec(dst + c + 32 * u, pack8(o));
+                    dk += part;
+                    st_vec(dst + c, pack8(o));
                 }
             }
-        }
-        if (grad_w) {
 #pragma unroll
-            for (int k = 0; k < KT; ++k) {
-                double v = dot[k];
-#pragma unroll
-                for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(kFull, v, d);
-                if (lane == k) {
-                    const int64_t f = (int64_t)t * KT + k;
-                    if (wdtype == MOE_DTYPE_F32) {
-                        static_cast<float*>(grad_w)[f] = __double2float_rn(v);
-                    } else {
-                        __nv_bfloat16 b = __double2bfloat16(v);
-                        static_cast<uint16_t*>(grad_w)[f] = *reinterpret_cast<uint16_t*>(&b);
-                    }
+            for (int d = 16; d > 0; d >>= 1) dk += __shfl_xor_sync(kFull, dk, d);
+            if (grad_w && lane == 0) {
+                const int64_t f = (int64_t)t * K + k;
+                if (wdtype == MOE_DTYPE_F32) {
+                    static_cast<float*>(grad_w)[f] = __double2float_rn(dk);
+                } else {
+                    __nv_bfloat16 b = __double2bfloat16(dk);
+                    static_cast<uint16_t*>(grad_w)[f] = *reinterpret_cast<uint16_t*>(&b);
                 }
             }
-        }
         }
     }
 
@@ -287,19 +292,138 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
     warp_status_or(status, bad);
 }
 
+// ------------------------------------------------ backward, slot-major ---
+//
+// One warp per token.  The row is walked in chunks of 32 lanes x U vectors;
+// per chunk, g is loaded once, then the slots k = 0..K-1 are visited in
+// order with D row chunks of y in flight (a ring): the dot product with g
+// accumulates in fp64 per slot (registers, across chunks), and the slot's
+// gradient chunk bf16_rn(w_k * g) is stored as a contiguous run.
+template <int KT, int U, int D>
+__global__ void __launch_bounds__(kBlock)
+combine_bwd_slots_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ rows,
+                         int64_t N_cap, const int32_t* __restrict__ r2f,
+                         const int32_t* __restrict__ f2r, const void* __restrict__ w, int wdtype,
+                         int T, int H, const int32_t* __restrict__ offsets, int E, int zero_pad,
+                         uint16_t* __restrict__ grad_rows, void* __restrict__ grad_w,
+                         int32_t* __restrict__ status) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n16 = H >> 3;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    int bad = 0;
+
+    for (int t = blockIdx.x * kWarps + warp; t < T; t += gridDim.x * kWarps) {
+        int myrow = -1;
+        float myw = 0.f;
+        if (lane < KT) {
+            const int64_t f = (int64_t)t * KT + lane;
+            int r = f2r[f];
+            if (r < 0 || (int64_t)r >= N_cap) {
+                bad |= MOE_ST_ROW_OOR;
+                r = -1;
+            } else {
+                myw = load_weight(w, wdtype, f);
+            }
+            myrow = r;
+        }
+        int rk[KT];
+        float wk[KT];
+        double dot[KT];
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+            rk[k] = __shfl_sync(kFull, myrow, k);
+            wk[k] = __shfl_sync(kFull, myw, k);
+            dot[k] = 0.0;
+        }
+        const uint4* gsrc = reinterpret_cast<const uint4*>(g + (size_t)t * H);
+        for (int c0 = 0; c0 < n16; c0 += 32 * U) {
+            const int v0 = c0 + lane;
+            uint4 gv[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) gv[u] = (v0 + 32 * u < n16) ? ld_stream(gsrc + v0 + 32 * u) : zero;
+            uint4 ring[D][U];
+#pragma unroll
+            for (int k = 0; k < D && k < KT; ++k) {
+                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[k] < 0 ? 0 : rk[k]) * H);
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    ring[k][u] = (rk[k] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
+            }
+#pragma unroll
+            for (int k = 0; k < KT; ++k) {
+                const int slot = k % D;
+                if (rk[k] >= 0) {
+                    uint4* dst = reinterpret_cast<uint4*>(grad_rows + (size_t)rk[k] * H);
+                    double part = 0.0;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        if (v0 + 32 * u >= n16) continue;
+                        float gf[8], yf[8], o[8];
+                        unpack8(gv[u], gf);
+                        unpack8(ring[slot][u], yf);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            part += (double)__fmul_rn(gf[i], yf[i]);   // exact: bf16 x bf16
+                            o[i] = __fmul_rn(wk[k], gf[i]);
+                        }
+                        st_vec(dst + v0 + 32 * u, pack8(o));
+                    }
+                    dot[k] += part;
+                }
+                if (k + D < KT) {
+                    const int kn = k + D;
+                    const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[kn] < 0 ? 0 : rk[kn]) * H);
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+                        ring[slot][u] = (rk[kn] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
+                }
+            }
+        }
+        if (grad_w) {
+#pragma unroll
+            for (int k = 0; k < KT; ++k) {
+                double v = dot[k];
+#pragma unroll
+                for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(kFull, v, d);
+                if (lane == k) {
+                    const int64_t f = (int64_t)t * KT + k;
+                    if (wdtype == MOE_DTYPE_F32) {
+                        static_cast<float*>(grad_w)[f] = __double2float_rn(v);
+                    } else {
+                        __nv_bfloat16 b = __double2bfloat16(v);
+                        static_cast<uint16_t*>(grad_w)[f] = *reinterpret_cast<uint16_t*>(&b);
+                    }
+                }
+            }
+        }
+    }
+
+    if (zero_pad) {
+        const int64_t N_pad = offsets[E];
+        const int64_t limit = N_pad < N_cap ? N_pad : N_cap;
+        const int64_t wstride = (int64_t)gridDim.x * kWarps * 32;
+        for (int64_t base = ((int64_t)blockIdx.x * kWarps + warp) * 32; base < limit; base += wstride) {
+            const int64_t row = base + lane;
+            const bool pad = row < limit && r2f[row] < 0;
+            unsigned m = __ballot_sync(kFull, pad);
+            while (m) {
+                const int b = __ffs(m) - 1;
+                m &= m - 1;
+                uint4* dst = reinterpret_cast<uint4*>(grad_rows + (size_t)(base + b) * H);
+                for (int c = lane; c < n16; c += 32) st_vec(dst + c, zero);
+            }
+        }
+    }
+    warp_status_or(status, bad);
+}
+
 // ------------------------------------------------------------ launchers ---
 
 template <bool V>
 static void launch_combine_t(int K, int grid, cudaStream_t st, const uint16_t* rows, int64_t N_cap,
                              const int32_t* r2f, const int32_t* f2r, const void* w, int wd, int T,
                              int H, uint16_t* out, int32_t* status) {
-    switch (K) {
-        case 1: combine_kernel<1, 8, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, K, H, out, status); break;
-        case 2: combine_kernel<2, 4, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, K, H, out, status); break;
-        case 4: combine_kernel<4, 2, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, K, H, out, status); break;
-        case 8: combine_kernel<8, 1, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, K, H, out, status); break;
-        default: combine_kernel<0, 2, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, K, H, out, status); break;
-    }
+    combine_kernel<2, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, K, H, out, status);
 }
 
 // Enough warps for one token each (up to 8 resident CTAs per SM), and, when a
@@ -315,10 +439,48 @@ static int grid_tokens_and_rows(int T, int64_t N_cap, bool sweep_rows) {
     return want < 1 ? 1 : (int)want;
 }
 
+template <bool V>
+static void launch_slots_t(int K, int grid, cudaStream_t st, const uint16_t* rows, int64_t N_cap,
+                           const int32_t* r2f, const int32_t* f2r, const void* w, int wd, int T,
+                           int H, uint16_t* out, int32_t* status) {
+    constexpr int U = MOE_COMBINE_U, D = MOE_COMBINE_D;
+    // Small K: wider chunks keep as many vectors in flight per lane.
+    switch (K) {
+        case 1: combine_slots_kernel<1, 4 * U, 1, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
+        case 2: combine_slots_kernel<2, 2 * U, 2, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
+        case 3: combine_slots_kernel<3, U, (D < 3 ? D : 3), V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
+        case 4: combine_slots_kernel<4, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
+        case 5: combine_slots_kernel<5, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
+        case 6: combine_slots_kernel<6, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
+        case 7: combine_slots_kernel<7, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
+        default: combine_slots_kernel<8, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
+    }
+}
+
 cudaError_t launch_combine(const uint16_t* rows, int64_t N_cap, const int32_t* row_to_flat,
                            const int32_t* flat_to_row, const void* weights, int weight_dtype,
                            int T, int K, int H, int validate, uint16_t* out, int32_t* status,
                            cudaStream_t stream) {
+    if (K <= 8) {
+        const int n16 = H >> 3;
+        const int u = K == 1 ? 4 * MOE_COMBINE_U : (K == 2 ? 2 * MOE_COMBINE_U : MOE_COMBINE_U);
+        const int chunks = (n16 + 32 * u - 1) / (32 * u);
+        const int64_t items = (int64_t)T * chunks;
+        const int cap = sm_count_current_device() * 8;
+        int64_t want = (items + kWarps - 1) / kWarps;
+        if (validate) {
+            const int64_t rw = (N_cap + kBlock - 1) / kBlock;
+            if (rw > want) want = rw;
+        }
+        const int grid = (int)(want > cap ? cap : (want < 1 ? 1 : want));
+        if (validate)
+            launch_slots_t<true>(K, grid, stream, rows, N_cap, row_to_flat, flat_to_row, weights,
+                                 weight_dtype, T, H, out, status);
+        else
+            launch_slots_t<false>(K, grid, stream, rows, N_cap, row_to_flat, flat_to_row, weights,
+                                  weight_dtype, T, H, out, status);
+        return cudaGetLastError();
+    }
     const int grid = grid_tokens_and_rows(T, N_cap, validate != 0);
     if (validate)
         launch_combine_t<true>(K, grid, stream, rows, N_cap, row_to_flat, flat_to_row, weights,
@@ -328,6 +490,10 @@ cudaError_t launch_combine(const uint16_t* rows, int64_t N_cap, const int32_t* r
                                 weight_dtype, T, H, out, status);
     return cudaGetLastError();
 }
+
+#define MOE_BWD_SLOT_ARGS                                                                      \
+    grad_out, rows, N_cap, row_to_flat, flat_to_row, weights, weight_dtype, T, H, expert_offsets,  \
+        E, zero_pad, grad_rows, grad_weights, status
 
 #define MOE_BWD_ARGS                                                                           \
     grad_out, rows, N_cap, row_to_flat, flat_to_row, weights, weight_dtype, T, K, H,           \
@@ -340,16 +506,17 @@ cudaError_t launch_combine_backward(const uint16_t* grad_out, const uint16_t* ro
                                     uint16_t* grad_rows, void* grad_weights, int32_t* status,
                                     cudaStream_t stream) {
     const int grid = grid_tokens_and_rows(T, N_cap, zero_pad != 0);
+    constexpr int U = MOE_COMBINE_U, D = MOE_COMBINE_D;
     switch (K) {
-        case 1: combine_bwd_kernel<1, 8><<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
-        case 2: combine_bwd_kernel<2, 4><<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
-        case 3: combine_bwd_kernel<3, 2><<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
-        case 4: combine_bwd_kernel<4, 2><<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
-        case 5: combine_bwd_kernel<5, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
-        case 6: combine_bwd_kernel<6, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
-        case 7: combine_bwd_kernel<7, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
-        case 8: combine_bwd_kernel<8, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
-        default: combine_bwd_kernel<0, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
+        case 1: combine_bwd_slots_kernel<1, 4 * U, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 2: combine_bwd_slots_kernel<2, 2 * U, 2><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 3: combine_bwd_slots_kernel<3, U, (D < 3 ? D : 3)><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 4: combine_bwd_slots_kernel<4, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 5: combine_bwd_slots_kernel<5, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 6: combine_bwd_slots_kernel<6, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 7: combine_bwd_slots_kernel<7, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 8: combine_bwd_slots_kernel<8, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        default: combine_bwd_kernel<<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
     }
     return cudaGetLastError();
 }

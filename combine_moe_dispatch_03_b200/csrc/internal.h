@@ -7,27 +7,33 @@
 
 namespace moe {
 
-// Layout workspace: [header | tile_base (E x n_tiles) | tile_tpr (n_tiles x R)
-// | expert_count (E)], each part 256-byte aligned.  Tiles are runs of at most
-// TT consecutive tokens that never straddle two source ranks' token blocks, so
-// per-rank sums are sums over whole tiles.  tile_base[e][j] first holds the
-// number of expert-e assignments in tile j, then (after the scan) the number
-// in all earlier tiles: the stable base of tile j inside expert e's group.
+// Layout workspace: [header | tile_base (E x n_tiles) | tile_tpr (R x n_tiles)
+// | expert_count (E) | in_rank (A = T*K, uint16)], each part 256-byte
+// aligned.  Tiles are runs of at most TT consecutive tokens that never
+// straddle two source ranks' token blocks, so per-rank sums are sums over
+// whole tiles.  tile_base[e][j] first holds the number of expert-e
+// assignments in tile j, then (after the scan) the number in all earlier
+// tiles: the stable base of tile j inside expert e's group.  in_rank[f] is
+// the number of earlier assignments of f's expert inside f's tile, so
+//     row(f) = expert_offsets[e] + tile_base[e][tile(t)] + in_rank[f].
 struct LayoutHeader {
     int64_t off_tile_base;     // byte offsets of the parts (so a reader needs no R)
     int64_t off_tile_tpr;
     int64_t off_expert_count;
+    int64_t off_in_rank;
     int32_t magic;
     int32_t T, K, E, R;
     int32_t TT;        // tokens per tile
     int32_t tpb;       // tiles per source block
     int32_t n_tiles;   // R * tpb
     uint32_t done;     // arrival counter of the scan kernel (self-resetting)
+    int32_t pad[7];
 };
-static_assert(sizeof(LayoutHeader) == 64, "header is 64 bytes");
+static_assert(sizeof(LayoutHeader) == 96, "header layout");
 
 constexpr int32_t kLayoutMagic = 0x4d6f4531;  // "MoE1"
-constexpr int kMaxTileAssign = 512;          // TT * K <= this
+constexpr int kMaxTileAssign = 512;          // TT * K <= this (16 warp chunks)
+constexpr int kMaxTileChunks = kMaxTileAssign / 32;
 
 struct Geometry {
     int TT, tpb, n_tiles;
@@ -53,15 +59,16 @@ inline Geometry layout_geometry(int T, int K, int R) {
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t tile_base, tile_tpr, expert_count, total;
+    size_t tile_base, tile_tpr, expert_count, in_rank, total;
 };
 
-inline WsLayout workspace_layout(int E, int R, int n_tiles) {
+inline WsLayout workspace_layout(int E, int R, int n_tiles, int64_t A) {
     WsLayout w;
     w.tile_base = align256(sizeof(LayoutHeader));
     w.tile_tpr = w.tile_base + align256(sizeof(int32_t) * (size_t)E * (size_t)n_tiles);
     w.expert_count = w.tile_tpr + align256(sizeof(int32_t) * (size_t)n_tiles * (size_t)R);
-    w.total = w.expert_count + align256(sizeof(int32_t) * (size_t)E);
+    w.in_rank = w.expert_count + align256(sizeof(int32_t) * (size_t)E);
+    w.total = w.in_rank + align256(sizeof(uint16_t) * (size_t)A);
     return w;
 }
 

@@ -6,24 +6,26 @@
 // token-group padding of its Attribution section.
 //
 // Assignment f = (t, k) of expert e goes to row
-//     off[e] + (assignments of e in earlier tiles) + (earlier in this tile)
-// which is the stable (expert, token, slot) order.  The first two terms come
-// from the layout workspace; the in-tile rank is computed by one warp walking
-// the tile's assignments in flat order, 32 at a time, with __match_any_sync
-// giving each lane the lanes that share its expert.
-//
-// Data movement (the cost: one read of x, K writes of every row): one warp per
-// token holds U 16-byte vectors per lane in registers and stores them to the
-// K destination rows, so x is read from HBM exactly once and every store is a
-// full, aligned, coalesced 512-byte warp transaction.  CTAs are persistent
-// over tiles (grid <= SMs x resident CTAs), then share the pad rows evenly.
+//     off[e] + (assignments of e in earlier tiles) + (earlier in its tile)
+// which is the stable (expert, token, slot) order.  All three terms are ready
+// in the layout workspace (the per-tile bases after the scan and the
+// in-tile ranks the histogram pass computed), so this is one streaming kernel:
+// one read of every token row, K writes of it, the two row maps, and the
+// pad rows.  Work is cut into equal warp items (4 KB row pieces) and strided
+// over a grid of several CTAs per SM, so every warp moves the same bytes.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
+// Grid-stride over warp items, all of one size: first (token, piece) items --
+// a piece is 32 lanes x U 16-byte vectors of the token's row, read once and
+// stored to the token's K rows -- then (pad row, piece) items.  The rows come
+// from the layout workspace: row(f) = off[e] + tile_base[e][tile(t)] +
+// in_rank[f]; the warp that handles piece 0 of a token also writes the
+// token's entries of both maps.  A final sweep marks the tail rows.
 template <int U>
-__global__ void __launch_bounds__(kBlock)
+__global__ void __launch_bounds__(kBlock, 4)
 permute_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ topk, int T, int K,
                int E, int H, const int32_t* __restrict__ offsets, const char* __restrict__ ws,
                int zero_pad, int64_t N_cap, uint16_t* __restrict__ xp,
@@ -32,139 +34,113 @@ permute_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ topk,
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int scratch[kWarps + 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
     const LayoutHeader* hdr = reinterpret_cast<const LayoutHeader*>(ws);
     if (hdr->magic != kLayoutMagic || hdr->T != T || hdr->K != K || hdr->E != E) {
         if (blockIdx.x == 0 && tid == 0) atomicOr(status, MOE_ST_LAYOUT_MISMATCH);
         return;
     }
     const int R = hdr->R, TT = hdr->TT, tpb = hdr->tpb, n_tiles = hdr->n_tiles;
+    const int Tb = T / R;
     const int32_t* tile_base = reinterpret_cast<const int32_t*>(ws + hdr->off_tile_base);
     const int32_t* ecount = reinterpret_cast<const int32_t*>(ws + hdr->off_expert_count);
+    const uint16_t* in_rank = reinterpret_cast<const uint16_t*>(ws + hdr->off_in_rank);
 
-    int* base = reinterpret_cast<int*>(smem_raw);   // [E+1]
-    int* eidx = base + (E + 1);                      // [TT*K]
-    int* rowi = eidx + TT * K;                       // [TT*K]
-
-    const int64_t N_pad = offsets[E];
-    if (blockIdx.x == 0 && tid == 0 && N_pad > N_cap) atomicOr(status, MOE_ST_CAPACITY);
-    const int Tb = T / R;
-    const int n16 = H >> 3;
-    int bad = 0;
-
-    for (int j = blockIdx.x; j < n_tiles; j += gridDim.x) {
-        const int s = j / tpb, i = j - s * tpb;
-        const int t0 = s * Tb + i * TT;
-        const int t1 = min(t0 + TT, (s + 1) * Tb);
-        const int ntok = t1 - t0, na = ntok * K;
-
-        for (int e = tid; e < E; e += kBlock) base[e] = offsets[e] + tile_base[(size_t)e * n_tiles + j];
-        for (int a = tid; a < na; a += kBlock) {
-            const int64_t v = topk[(int64_t)t0 * K + a];
-            eidx[a] = (v >= 0 && v < E) ? (int)v : -1;
-        }
-        __syncthreads();
-
-        if (warp == 0) {
-            const unsigned lt = lanemask_lt();
-            for (int c0 = 0; c0 < na; c0 += 32) {
-                const int a = c0 + lane;
-                const int e = (a < na) ? eidx[a] : -1;
-                const int key = (e >= 0) ? e : (-1 - lane);
-                const unsigned peers = __match_any_sync(kFull, key);
-                int row = -1;
-                if (e >= 0) row = base[e] + __popc(peers & lt);
-                __syncwarp();
-                if (e >= 0 && lane == __ffs(peers) - 1) base[e] += __popc(peers);
-                __syncwarp();
-                if (a < na) {
-                    const int64_t f = (int64_t)t0 * K + a;
-                    const bool placed = (row >= 0) && ((int64_t)row < N_cap);
-                    rowi[a] = placed ? row : -1;
-                    f2r[f] = placed ? row : -1;
-                    if (placed) r2f[row] = (int32_t)f;
-                    if (e < 0) bad |= MOE_ST_EXPERT_OOR;
-                    else if (!placed) bad |= MOE_ST_CAPACITY;
-                }
-            }
-        }
-        __syncthreads();
-
-        // ---- copies: one warp per token, K stores per loaded vector ----
-        for (int q = warp; q < ntok; q += kWarps) {
-            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(t0 + q) * H);
-            const int myrow = (lane < K) ? rowi[q * K + lane] : -1;
-            // Warp-uniform trip count (the shuffles below need all 32 lanes);
-            // accesses past the row end are predicated off.
-            for (int c0 = 0; c0 < n16; c0 += 32 * U) {
-                const int c = c0 + lane;
-                uint4 v[U];
-#pragma unroll
-                for (int u = 0; u < U; ++u)
-                    if (c + 32 * u < n16) v[u] = ld_stream(src + c + 32 * u);
-                for (int k = 0; k < K; ++k) {
-                    const int r = __shfl_sync(kFull, myrow, k);
-                    if (r < 0) continue;
-                    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * H);
-#pragma unroll
-                    for (int u = 0; u < U; ++u)
-                        if (c + 32 * u < n16) st_vec(dst + c + 32 * u, v[u]);
-                }
-            }
-        }
-        __syncthreads();
-    }
-    warp_status_or(status, bad);
-
-    // ---- pad rows [off[e] + c_e, off[e+1]) and the tail [N_pad, N_cap) ----
-    int* padstart = base;  // [E+1] exclusive prefix of pad rows per expert
-    for (int e = tid; e < E; e += kBlock) padstart[e] = (offsets[e + 1] - offsets[e]) - ecount[e];
+    int* off = reinterpret_cast<int*>(smem_raw);   // [E+1]
+    int* padstart = off + (E + 1);                  // [E+1]
+    for (int e = tid; e <= E; e += kBlock) off[e] = offsets[e];
+    __syncthreads();
+    for (int e = tid; e < E; e += kBlock) padstart[e] = (off[e + 1] - off[e]) - ecount[e];
     __syncthreads();
     const int P = block_exclusive_scan<MOE_MAX_E / kBlock>(padstart, E, scratch);
     if (tid == 0) padstart[E] = P;
     __syncthreads();
+    const int64_t N_pad = off[E];
+    if (blockIdx.x == 0 && tid == 0 && N_pad > N_cap) atomicOr(status, MOE_ST_CAPACITY);
 
-    const int gwarp = blockIdx.x * kWarps + warp;
-    const int nwarps = gridDim.x * kWarps;
+    const int n16 = H >> 3;
+    const int pieces = (n16 + 32 * U - 1) / (32 * U);
+    const int64_t tok_items = (int64_t)T * pieces;
+    const int64_t n_items = tok_items + (int64_t)P * pieces;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    for (int q = gwarp; q < P; q += nwarps) {
-        const int e = upper_index(padstart, E + 1, q);
-        const int64_t row = (int64_t)offsets[e] + ecount[e] + (q - padstart[e]);
-        if (row < 0 || row >= N_cap) continue;
-        if (lane == 0) r2f[row] = -1;
-        if (zero_pad) {
+    int bad = 0;
+
+    for (int64_t item = (int64_t)blockIdx.x * kWarps + warp; item < n_items;
+         item += (int64_t)gridDim.x * kWarps) {
+        if (item < tok_items) {
+            const int64_t t = item / pieces;
+            const int p = (int)(item - t * pieces);
+            const int v0 = p * 32 * U + lane;
+            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+            uint4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) v[u] = (v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
+            int myrow = -1;
+            if (lane < K) {
+                const int64_t f = t * K + lane;
+                const int64_t e = topk[f];
+                if (e >= 0 && e < E) {
+                    const int s = (int)(t / Tb);
+                    const int jt = s * tpb + (int)(t - (int64_t)s * Tb) / TT;
+                    const int64_t row = (int64_t)off[e] + tile_base[(size_t)e * n_tiles + jt] + in_rank[f];
+                    if (row >= 0 && row < N_cap) myrow = (int)row;
+                    else if (p == 0) bad |= MOE_ST_CAPACITY;
+                } else if (p == 0) {
+                    bad |= MOE_ST_EXPERT_OOR;
+                }
+                if (p == 0) {
+                    f2r[f] = myrow;
+                    if (myrow >= 0) r2f[myrow] = (int32_t)f;
+                }
+            }
+            for (int k = 0; k < K; ++k) {
+                const int r = __shfl_sync(kFull, myrow, k);
+                if (r < 0) continue;
+                uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * H);
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (v0 + 32 * u < n16) st_vec(dst + v0 + 32 * u, v[u]);
+            }
+        } else {
+            const int64_t pi = item - tok_items;
+            const int q = (int)(pi / pieces);
+            const int p = (int)(pi - (int64_t)q * pieces);
+            const int v0 = p * 32 * U + lane;
+            const int e = upper_index(padstart, E + 1, q);
+            const int64_t row = (int64_t)off[e] + ecount[e] + (q - padstart[e]);
+            if (row < 0 || row >= N_cap) continue;
+            if (p == 0 && lane == 0) r2f[row] = -1;
+            if (!zero_pad) continue;
             uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * H);
-            for (int c = lane; c < n16; c += 32) st_vec(dst + c, zero);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (v0 + 32 * u < n16) st_vec(dst + v0 + 32 * u, zero);
         }
     }
-    const int64_t gtid = (int64_t)blockIdx.x * kBlock + tid;
+    warp_status_or(status, bad);
+
     const int64_t tail0 = N_pad > 0 ? N_pad : 0;
-    for (int64_t row = tail0 + gtid; row < N_cap; row += (int64_t)gridDim.x * kBlock) r2f[row] = -1;
+    for (int64_t row = tail0 + (int64_t)blockIdx.x * kBlock + tid; row < N_cap;
+         row += (int64_t)gridDim.x * kBlock)
+        r2f[row] = -1;
 }
 
 cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
                            const int32_t* expert_offsets, const void* workspace, int zero_pad,
                            int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat,
                            int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
-    // The tile geometry and the workspace parts are read from the header on
-    // the device, so R is not an argument.  Host-side bounds: every tile holds
-    // at least one token (n_tiles <= T), and the cap TT <= T/R only shrinks
-    // TT as R grows, so TT(R = 1) bounds the shared-memory tile buffers.
+    // Enough CTAs to fill every SM several times over; the kernel strides
+    // over its uniform items (token pieces, then pad-row pieces <= N_cap - A).
+    constexpr int U = 8;
     const int sms = sm_count_current_device();
-    int grid = sms * 4;
-    if (grid > T) grid = T;
+    const int n16 = H >> 3;
+    const int64_t pieces = (n16 + 32 * U - 1) / (32 * U);
+    const int64_t items = ((int64_t)T + (N_cap - (int64_t)T * K)) * pieces;
+    int64_t grid = (items + kWarps - 1) / kWarps;
+    if (grid > (int64_t)sms * 8) grid = (int64_t)sms * 8;
     if (grid < 1) grid = 1;
-    const int TTmax = layout_geometry(T, K, 1).TT;
-    const size_t smem = sizeof(int) * ((size_t)E + 1 + 2 * (size_t)TTmax * K);
-    const char* ws = static_cast<const char*>(workspace);
-    if (H >= 4096)
-        permute_kernel<4><<<grid, kBlock, smem, stream>>>(x, topk_idx, T, K, E, H, expert_offsets,
-                                                          ws, zero_pad, N_cap, x_perm, row_to_flat,
-                                                          flat_to_row, status);
-    else
-        permute_kernel<8><<<grid, kBlock, smem, stream>>>(x, topk_idx, T, K, E, H, expert_offsets,
-                                                          ws, zero_pad, N_cap, x_perm, row_to_flat,
-                                                          flat_to_row, status);
+    permute_kernel<U><<<(int)grid, kBlock, sizeof(int) * 2 * ((size_t)E + 1), stream>>>(
+        x, topk_idx, T, K, E, H, expert_offsets, static_cast<const char*>(workspace), zero_pad,
+        N_cap, x_perm, row_to_flat, flat_to_row, status);
     return cudaGetLastError();
 }
 

@@ -23,7 +23,8 @@ ST_CAPACITY = 2
 ST_ROW_OOR = 4
 ST_COVERAGE = 8
 ST_LAYOUT_MISMATCH = 16
-STATUS_BITS = (ST_EXPERT_OOR, ST_CAPACITY, ST_ROW_OOR, ST_COVERAGE, ST_LAYOUT_MISMATCH)
+ST_TIMEOUT = 32
+STATUS_BITS = (ST_EXPERT_OOR, ST_CAPACITY, ST_ROW_OOR, ST_COVERAGE, ST_LAYOUT_MISMATCH, ST_TIMEOUT)
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1

@@ -26,25 +26,28 @@ struct LayoutHeader {
     int32_t TT;        // tokens per tile
     int32_t tpb;       // tiles per source block
     int32_t n_tiles;   // R * tpb
-    uint32_t done;     // arrival counter of the scan kernel (self-resetting)
+    uint32_t done;     // arrival counter of the layout kernel (zeroed before each launch)
     int32_t pad[7];
 };
 static_assert(sizeof(LayoutHeader) == 96, "header layout");
 
 constexpr int32_t kLayoutMagic = 0x4d6f4531;  // "MoE1"
-constexpr int kMaxTileAssign = 512;          // TT * K <= this (16 warp chunks)
+constexpr int kMaxTileAssign = 1024;          // TT * K <= this (32 warp chunks)
 constexpr int kMaxTileChunks = kMaxTileAssign / 32;
 
 struct Geometry {
     int TT, tpb, n_tiles;
 };
 
-// Tile geometry: about 4 tiles per SM of a 148-SM B200 for the large configs,
-// at most kMaxTileAssign assignments per tile.  A pure function of the sizes,
-// so the workspace size is known before any device is touched.
+// Tile geometry: about one tile per SM of a 148-SM B200 (the layout kernel
+// runs one 1024-thread CTA per tile), at most kMaxTileAssign assignments per
+// tile.  A pure function of the sizes, so the workspace size is known before
+// any device is touched.
 inline Geometry layout_geometry(int T, int K, int R) {
     const int Tb = R > 0 ? T / R : 0;
-    int tt = (T + 591) / 592;
+    int per_block = R > 0 ? 148 / R : 1;          // tiles per source block, <= 148 in all
+    if (per_block < 1) per_block = 1;
+    int tt = (Tb + per_block - 1) / per_block;
     int cap = kMaxTileAssign / K;
     if (tt > cap) tt = cap;
     if (tt < 1) tt = 1;

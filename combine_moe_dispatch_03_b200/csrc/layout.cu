@@ -4,233 +4,331 @@
 // "Derive AutoEP rank splits from the per-expert count exchange", Redundancy;
 // the group alignment of the DeepSpeed AutoEP base PR, Attribution).
 //
-// Two launches, no host synchronisation:
-//   layout_hist_kernel  one CTA per tile of <= TT tokens: per-expert counts of
-//                       the tile (warp-aggregated shared-memory histogram),
-//                       is_token_in_rank rows, distinct tokens per rank.
-//   layout_scan_kernel  one warp per expert: exclusive scan of the expert's
-//                       tile counts (its stable per-tile bases, read back by
-//                       the permute) and its per-source-block counts; one warp
-//                       per destination rank does the same for the per-tile
-//                       distinct-token counts (tokens_per_rank); the last CTA
-//                       to arrive then builds the padded offsets and splits
-//                       from the other CTAs' results (arrival counter, no
-//                       waiting).
+// One kernel, no host synchronisation.  Tiles of <= TT consecutive tokens
+// (at most 148, never straddling a source rank's token block) each get a
+// 1024-thread CTA:
+//   phase 1 (every CTA, its tile): each warp ranks whole 32-assignment chunks
+//     in flat order with __match_any_sync (lanes sharing an expert find each
+//     other; a lane's rank is the number of lower lanes of its expert); the
+//     chunk counts give every assignment's stable in-tile rank and the tile's
+//     per-expert count; token rank masks give is_token_in_rank and the tile's
+//     distinct tokens per destination rank.
+//   phase 2: one warp per row of per-tile counts -- experts, then destination
+//     ranks -- scans the row over the tiles (the expert rows are rewritten in
+//     place as the per-tile stable bases the permute reads) and sums it per
+//     source block (count matrix, tokens_per_rank).
+//   phase 3: padded exclusive offsets and splits.
+// When every tile's CTA fits on the GPU at once the launch is cooperative:
+// phases are separated by two grid barriers (bounded spins on a counter that
+// record MOE_ST_TIMEOUT instead of hanging) and phase 2 is spread over every
+// warp of the grid.  Otherwise the last CTA to arrive (an arrival counter, no
+// waiting) runs phases 2 and 3 alone.  The counter lives in the workspace
+// header and is zeroed by a 4-byte memset enqueued just before the kernel.
 //
-// Bytes: reads topk_idx once (8*A), writes [T,R] flags and O(E*tiles) ints.
+// Bytes: reads topk_idx once (8*A), writes the [T,R] flags, in-tile ranks
+// (2*A) and O((E+R) * tiles) ints.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
-__global__ void __launch_bounds__(kBlock)
-layout_hist_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, Geometry geo,
-                   uint8_t* __restrict__ itr, char* __restrict__ ws, WsLayout wl,
-                   int32_t* __restrict__ status) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned long long* tokmask = reinterpret_cast<unsigned long long*>(smem_raw);  // [TT]
-    int* eidx = reinterpret_cast<int*>(tokmask + geo.TT);                          // [TT*K]
-    uint16_t* crank = reinterpret_cast<uint16_t*>(eidx + geo.TT * K);               // [TT*K]
-    uint16_t* cnt = crank + ((geo.TT * K + 1) & ~1);                                // [chunks][E]
+constexpr int kLThreads = 1024;
+constexpr int kLWarps = kLThreads / 32;
+constexpr size_t kLayoutSmemMax = 200 * 1024;   // staging limit for phase 2
 
-    const int j = blockIdx.x;
+// In-place exclusive scan of n <= kLThreads ints in shared memory by a
+// 1024-thread CTA; returns the total.  `scratch` holds kLWarps + 1 ints.
+__device__ int block_exclusive_scan_1024(int* data, int n, int* scratch) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (j == 0 && tid == 0) {
-        LayoutHeader* h = reinterpret_cast<LayoutHeader*>(ws);
-        h->off_tile_base = (int64_t)wl.tile_base;
-        h->off_tile_tpr = (int64_t)wl.tile_tpr;
-        h->off_expert_count = (int64_t)wl.expert_count;
-        h->off_in_rank = (int64_t)wl.in_rank;
-        h->magic = kLayoutMagic;
-        h->T = T; h->K = K; h->E = E; h->R = R;
-        h->TT = geo.TT; h->tpb = geo.tpb; h->n_tiles = geo.n_tiles;
-        h->done = 0u;
+    const int v = tid < n ? data[tid] : 0;
+    int incl = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int x = __shfl_up_sync(kFull, incl, d);
+        if (lane >= d) incl += x;
     }
-    if (j >= geo.n_tiles) return;
-
-    int32_t* tile_base = reinterpret_cast<int32_t*>(ws + wl.tile_base);
-    int32_t* tile_tpr = reinterpret_cast<int32_t*>(ws + wl.tile_tpr);
-    uint16_t* in_rank = reinterpret_cast<uint16_t*>(ws + wl.in_rank);
-    const int Tb = T / R, El = E / R;
-    const int s = j / geo.tpb, i = j - s * geo.tpb;
-    const int t0 = s * Tb + i * geo.TT;
-    const int t1 = min(t0 + geo.TT, (s + 1) * Tb);
-    const int ntok = t1 - t0, na = ntok * K;
-    const int nchunks = (na + 31) / 32;
-
-    for (int q = tid; q < nchunks * E; q += kBlock) cnt[q] = 0;
-    for (int q = tid; q < ntok; q += kBlock) tokmask[q] = 0ull;
+    if (lane == 31) scratch[warp] = incl;
     __syncthreads();
-
-    // Every warp ranks whole 32-assignment chunks of the tile (flat order):
-    // lanes sharing an expert find each other with __match_any_sync; a
-    // lane's rank inside its chunk is the number of lower lanes of the same
-    // expert, and the chunk's count per expert is written by its leader.
-    int bad = 0;
-    const unsigned lt = lanemask_lt();
-    for (int c = warp; c < nchunks; c += kWarps) {
-        const int a = c * 32 + lane;
-        int key = -1 - lane;
-        if (a < na) {
-            const int64_t e = topk[(int64_t)t0 * K + a];
-            if (e >= 0 && e < E) key = (int)e; else bad = MOE_ST_EXPERT_OOR;
-            eidx[a] = key >= 0 ? key : -1;
+    if (warp == 0) {
+        const int w = scratch[lane];
+        int wi = w;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int x = __shfl_up_sync(kFull, wi, d);
+            if (lane >= d) wi += x;
         }
-        const unsigned peers = __match_any_sync(kFull, key);
-        if (key >= 0) {
-            crank[a] = (uint16_t)__popc(peers & lt);
-            if (lane == __ffs(peers) - 1) cnt[c * E + key] = (uint16_t)__popc(peers);
-            atomicOr(&tokmask[a / K], 1ull << (key / El));
-        }
+        scratch[lane] = wi - w;
+        if (lane == 31) scratch[kLWarps] = wi;
     }
-    warp_status_or(status, bad);
     __syncthreads();
-
-    // In-tile stable rank = assignments of the same expert in earlier chunks
-    // + rank inside the chunk.
-    uint16_t* out_rank = in_rank + (size_t)t0 * K;
-    for (int a = tid; a < na; a += kBlock) {
-        const int e = eidx[a];
-        if (e < 0) { out_rank[a] = 0xFFFFu; continue; }
-        int before = 0;
-        for (int c = 0; c < a / 32; ++c) before += cnt[c * E + e];
-        out_rank[a] = (uint16_t)(before + crank[a]);
-    }
-    for (int e = tid; e < E; e += kBlock) {
-        int total = 0;
-        for (int c = 0; c < nchunks; ++c) total += cnt[c * E + e];
-        tile_base[(size_t)e * geo.n_tiles + j] = total;
-    }
-    uint8_t* itr_tile = itr + (size_t)t0 * R;
-    for (int idx = tid; idx < ntok * R; idx += kBlock) {
-        const int q = idx / R, r = idx - q * R;
-        itr_tile[idx] = (uint8_t)((tokmask[q] >> r) & 1ull);
-    }
-    for (int r = tid; r < R; r += kBlock) {
-        int n = 0;
-        for (int q = 0; q < ntok; ++q) n += (int)((tokmask[q] >> r) & 1ull);
-        tile_tpr[(size_t)r * geo.n_tiles + j] = n;     // rank-major, like tile_base
-    }
+    if (tid < n) data[tid] = scratch[warp] + incl - v;
+    const int total = scratch[kLWarps];
+    __syncthreads();
+    return total;
 }
 
-constexpr int kScanBatch = 32;  // 32-tile chunks loaded per batch (independent loads)
+constexpr uint64_t kBarrierLimitNs = 2000000000ull;   // 2 s
 
-__global__ void __launch_bounds__(kBlock)
-layout_scan_kernel(int E, int R, int align, Geometry geo, int32_t* __restrict__ tokens_per_expert,
-                   int32_t* __restrict__ counts, int32_t* __restrict__ splits,
-                   int32_t* __restrict__ tokens_per_rank, int32_t* __restrict__ offsets,
-                   char* __restrict__ ws, WsLayout wl) {
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Grid barrier for a cooperative launch: every CTA adds one arrival to
+// `bar` (zeroed before the launch) and waits until `target` arrivals.  The
+// wait is bounded; returns false if it gave up.
+__device__ bool grid_barrier(unsigned* bar, unsigned target) {
+    __shared__ int ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(bar, 1u);
+        const uint64_t t0 = global_timer_ns();
+        int good = 1;
+        for (;;) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+            if (v >= target) break;
+            if (global_timer_ns() - t0 > kBarrierLimitNs) { good = 0; break; }
+            __nanosleep(64);
+        }
+        __threadfence();
+        ok = good;
+    }
+    __syncthreads();
+    return ok != 0;
+}
+
+// Phase 2 for one row p of per-tile counts (all 32 lanes): exclusive scan
+// over the tiles with lane-contiguous segments, written back in place for
+// expert rows; block sums into the count matrix / tokens_per_rank.  `rows`
+// is the row in shared memory when staged, else nullptr (global).
+struct RowOut {
+    int total;
+};
+__device__ RowOut scan_row(int p, int E, int R, const Geometry& geo, int32_t* tile_base,
+                           int32_t* tile_tpr, int* smem_row, int* bs, int32_t* counts,
+                           int32_t* tokens_per_rank) {
+    const int lane = threadIdx.x & 31;
+    const int n_tiles = geo.n_tiles, El = E / R;
+    const bool is_expert = p < E;
+    int32_t* rowg = is_expert ? tile_base + (size_t)p * n_tiles
+                              : tile_tpr + (size_t)(p - E) * n_tiles;
+    int* rows = smem_row ? smem_row : rowg;
+    for (int q = lane; q <= R; q += 32) bs[q] = 0;
+    __syncwarp();
+    const int seg = (n_tiles + 31) / 32;
+    const int j0 = min(lane * seg, n_tiles), j1 = min(j0 + seg, n_tiles);
+    int local = 0;
+    for (int jj = j0; jj < j1; ++jj) local += smem_row ? rows[jj] : __ldcg(rowg + jj);
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int x = __shfl_up_sync(kFull, incl, d);
+        if (lane >= d) incl += x;
+    }
+    const int total = __shfl_sync(kFull, incl, 31);
+    int run = incl - local;
+    for (int jj = j0; jj < j1; ++jj) {
+        const int v = smem_row ? rows[jj] : __ldcg(rowg + jj);
+        if (is_expert) rows[jj] = run;
+        if (jj % geo.tpb == 0) bs[jj / geo.tpb] = run;
+        run += v;
+    }
+    __syncwarp();
+    if (lane == 0) bs[R] = total;
+    __syncwarp();
+    if (is_expert) {
+        const int r = p / El, el = p - r * El;
+        for (int sb = lane; sb < R; sb += 32)
+            counts[((size_t)sb * R + r) * El + el] = bs[sb + 1] - bs[sb];
+    } else {
+        const int r = p - E;
+        for (int sb = lane; sb < R; sb += 32)
+            tokens_per_rank[(size_t)sb * R + r] = bs[sb + 1] - bs[sb];
+    }
+    __syncwarp();
+    RowOut o;
+    o.total = total;
+    return o;
+}
+
+__global__ void __launch_bounds__(kLThreads, 1)
+layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int align,
+              Geometry geo, int32_t* __restrict__ tokens_per_expert, int32_t* __restrict__ counts,
+              int32_t* __restrict__ splits, int32_t* __restrict__ tokens_per_rank,
+              uint8_t* __restrict__ itr, int32_t* __restrict__ offsets, char* __restrict__ ws,
+              WsLayout wl, int32_t* __restrict__ status, int coop, int staged) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    int* sm = reinterpret_cast<int*>(smem_raw);
-    __shared__ int scratch[kWarps + 1];
+    __shared__ int scratch[kLWarps + 1];
     __shared__ int am_last;
-
+    const int j = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int El = E / R;
+    const int Tb = R > 0 ? T / R : 0, El = E / R;
     const int n_tiles = geo.n_tiles;
     int32_t* tile_base = reinterpret_cast<int32_t*>(ws + wl.tile_base);
     int32_t* tile_tpr = reinterpret_cast<int32_t*>(ws + wl.tile_tpr);
     int32_t* expert_count = reinterpret_cast<int32_t*>(ws + wl.expert_count);
+    uint16_t* in_rank = reinterpret_cast<uint16_t*>(ws + wl.in_rank);
     LayoutHeader* hdr = reinterpret_cast<LayoutHeader*>(ws);
 
-    // ---- one warp per row of per-tile counts: rows 0..E-1 are experts, rows
-    // E..E+R-1 are destination ranks (distinct tokens per tile).  Each warp
-    // computes the exclusive scan of its row over the tiles (written back in
-    // place for experts: the stable per-tile bases the permute reads) and the
-    // sum over each source block's tiles.  Loads come in batches of
-    // kScanBatch coalesced 32-tile chunks, all issued before they are used.
-    int* bstart = sm + warp * (R + 1);
-    const int p = blockIdx.x * kWarps + warp;
-    if (p < E + R) {
-        const bool is_expert = p < E;
-        int32_t* rowp = is_expert ? tile_base + (size_t)p * n_tiles
-                                  : tile_tpr + (size_t)(p - E) * n_tiles;
-        for (int q = lane; q <= R; q += 32) bstart[q] = 0;
-        __syncwarp();
-        int running = 0;
-        for (int c0 = 0; c0 < n_tiles; c0 += 32 * kScanBatch) {
-            int v[kScanBatch];
-#pragma unroll
-            for (int b = 0; b < kScanBatch; ++b) {
-                const int jj = c0 + b * 32 + lane;
-                v[b] = (jj < n_tiles) ? rowp[jj] : 0;
+    if (j == 0 && tid == 0) {
+        hdr->off_tile_base = (int64_t)wl.tile_base;
+        hdr->off_tile_tpr = (int64_t)wl.tile_tpr;
+        hdr->off_expert_count = (int64_t)wl.expert_count;
+        hdr->off_in_rank = (int64_t)wl.in_rank;
+        hdr->magic = kLayoutMagic;
+        hdr->T = T; hdr->K = K; hdr->E = E; hdr->R = R;
+        hdr->TT = geo.TT; hdr->tpb = geo.tpb; hdr->n_tiles = n_tiles;
+    }
+
+    // ------------------------------------------------- phase 1: one tile ---
+    if (j < n_tiles) {
+        unsigned long long* tokmask = reinterpret_cast<unsigned long long*>(smem_raw);  // [TT]
+        int* eidx = reinterpret_cast<int*>(tokmask + geo.TT);                          // [TT*K]
+        uint16_t* crank = reinterpret_cast<uint16_t*>(eidx + geo.TT * K);               // [TT*K]
+        uint16_t* cnt = crank + ((geo.TT * K + 1) & ~1);                                // [chunks][E]
+        const int s = j / geo.tpb, i = j - s * geo.tpb;
+        const int t0 = s * Tb + i * geo.TT;
+        const int t1 = min(t0 + geo.TT, (s + 1) * Tb);
+        const int ntok = t1 - t0, na = ntok * K;
+        const int nchunks = (na + 31) / 32;
+
+        for (int q = tid; q < nchunks * E; q += kLThreads) cnt[q] = 0;
+        for (int q = tid; q < ntok; q += kLThreads) tokmask[q] = 0ull;
+        __syncthreads();
+
+        int bad = 0;
+        const unsigned lt = lanemask_lt();
+        for (int c = warp; c < nchunks; c += kLWarps) {
+            const int a = c * 32 + lane;
+            int key = -1 - lane;
+            if (a < na) {
+                const int64_t e = topk[(int64_t)t0 * K + a];
+                if (e >= 0 && e < E) key = (int)e; else bad = MOE_ST_EXPERT_OOR;
+                eidx[a] = key >= 0 ? key : -1;
             }
-#pragma unroll
-            for (int b = 0; b < kScanBatch; ++b) {
-                int incl = v[b];
-#pragma unroll
-                for (int d = 1; d < 32; d <<= 1) {
-                    const int n = __shfl_up_sync(kFull, incl, d);
-                    if (lane >= d) incl += n;
-                }
-                const int jj = c0 + b * 32 + lane;
-                const int excl = running + incl - v[b];
-                if (jj < n_tiles) {
-                    if (is_expert) rowp[jj] = excl;
-                    if (jj % geo.tpb == 0) bstart[jj / geo.tpb] = excl;
-                }
-                running += __shfl_sync(kFull, incl, 31);
+            const unsigned peers = __match_any_sync(kFull, key);
+            if (key >= 0) {
+                crank[a] = (uint16_t)__popc(peers & lt);
+                if (lane == __ffs(peers) - 1) cnt[c * E + key] = (uint16_t)__popc(peers);
+                atomicOr(&tokmask[a / K], 1ull << (key / El));
             }
         }
-        __syncwarp();
-        if (lane == 0) bstart[R] = running;
-        __syncwarp();
-        if (is_expert) {
-            const int r = p / El, el = p - r * El;
-            for (int sb = lane; sb < R; sb += 32)
-                counts[((size_t)sb * R + r) * El + el] = bstart[sb + 1] - bstart[sb];
-            if (lane == 0) {
-                tokens_per_expert[p] = running;
-                expert_count[p] = running;
-            }
-        } else {
-            const int r = p - E;
-            for (int sb = lane; sb < R; sb += 32)
-                tokens_per_rank[(size_t)sb * R + r] = bstart[sb + 1] - bstart[sb];
+        warp_status_or(status, bad);
+        __syncthreads();
+
+        // In-tile stable rank = same-expert assignments in earlier chunks +
+        // rank inside the chunk.
+        uint16_t* out_rank = in_rank + (size_t)t0 * K;
+        for (int a = tid; a < na; a += kLThreads) {
+            const int e = eidx[a];
+            if (e < 0) { out_rank[a] = 0xFFFFu; continue; }
+            int before = 0;
+            for (int c = 0; c < a / 32; ++c) before += cnt[c * E + e];
+            out_rank[a] = (uint16_t)(before + crank[a]);
+        }
+        for (int e = tid; e < E; e += kLThreads) {
+            int total = 0;
+            for (int c = 0; c < nchunks; ++c) total += cnt[c * E + e];
+            tile_base[(size_t)e * n_tiles + j] = total;
+        }
+        uint8_t* itr_tile = itr + (size_t)t0 * R;
+        for (int idx = tid; idx < ntok * R; idx += kLThreads) {
+            const int q = idx / R, r = idx - q * R;
+            itr_tile[idx] = (uint8_t)((tokmask[q] >> r) & 1ull);
+        }
+        for (int r = tid; r < R; r += kLThreads) {
+            int n = 0;
+            for (int q = 0; q < ntok; ++q) n += (int)((tokmask[q] >> r) & 1ull);
+            tile_tpr[(size_t)r * n_tiles + j] = n;     // rank-major, like tile_base
         }
     }
 
-    // ---- the last CTA to arrive finishes the cross-expert parts ----
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) am_last = (atomicAdd(&hdr->done, 1u) == gridDim.x - 1);
-    __syncthreads();
-    if (!am_last) return;
-    __threadfence();
+    unsigned* counter = &hdr->done;
+    int* bstart = reinterpret_cast<int*>(smem_raw);   // [kLWarps][R+1]
+    int* ctot = bstart + kLWarps * (R + 1);            // [E]
+    int* acc_splits = ctot + E;                        // [R*R]
+    int* mat = acc_splits + R * R;                     // [E+R][n_tiles] when staged
+    int* bs = bstart + warp * (R + 1);
+    const int nrows = E + R;
 
-    int* padded = sm;            // [E]
-    int* acc_splits = sm + E;    // [R*R]
-    for (int q = tid; q < E; q += kBlock) {
-        const int c = __ldcg(expert_count + q);
-        padded[q] = ((c + align - 1) / align) * align;
+    if (coop) {
+        // ---------------------- cooperative: phase 2 over the whole grid ---
+        if (!grid_barrier(counter, gridDim.x)) {
+            if (tid == 0) atomicOr(status, MOE_ST_TIMEOUT);
+            return;
+        }
+        for (int p = j * kLWarps + warp; p < nrows; p += gridDim.x * kLWarps) {
+            const RowOut o = scan_row(p, E, R, geo, tile_base, tile_tpr, nullptr, bs, counts,
+                                      tokens_per_rank);
+            if (p < E && lane == 0) {
+                tokens_per_expert[p] = o.total;
+                expert_count[p] = o.total;
+            }
+        }
+        if (!grid_barrier(counter, 2u * gridDim.x)) {
+            if (tid == 0) atomicOr(status, MOE_ST_TIMEOUT);
+            return;
+        }
+        if (j != 0) return;
+        // phase 3 inputs from global memory
+        for (int q = tid; q < R * R; q += kLThreads) acc_splits[q] = 0;
+        if (tid < E) ctot[tid] = __ldcg(expert_count + tid);
+        __syncthreads();
+        const int n = R * E;
+        for (int q = tid; q < n; q += kLThreads) {
+            const int v = __ldcg(counts + q);
+            if (v) atomicAdd(&acc_splits[q / El], v);
+        }
+        __syncthreads();
+    } else {
+        // ------------------- the last CTA to arrive runs phases 2 and 3 ---
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) am_last = (atomicAdd(counter, 1u) == gridDim.x - 1);
+        __syncthreads();
+        if (!am_last) return;
+        __threadfence();
+        for (int q = tid; q < R * R; q += kLThreads) acc_splits[q] = 0;
+        if (staged) {
+            // Stage the whole count matrix (independent coalesced loads).
+            const int ne = E * n_tiles, nr = R * n_tiles;
+            for (int q = tid; q < ne; q += kLThreads) mat[q] = __ldcg(tile_base + q);
+            for (int q = tid; q < nr; q += kLThreads) mat[ne + q] = __ldcg(tile_tpr + q);
+        }
+        __syncthreads();
+        for (int p = warp; p < nrows; p += kLWarps) {
+            const RowOut o = scan_row(p, E, R, geo, tile_base, tile_tpr,
+                                      staged ? mat + (size_t)p * n_tiles : nullptr, bs, counts,
+                                      tokens_per_rank);
+            if (p < E) {
+                const int r = p / El, el = p - r * El;
+                for (int sb = lane; sb < R; sb += 32)
+                    atomicAdd(&acc_splits[sb * R + r], bs[sb + 1] - bs[sb]);
+                if (lane == 0) {
+                    tokens_per_expert[p] = o.total;
+                    expert_count[p] = o.total;
+                    ctot[p] = o.total;
+                }
+            }
+            __syncwarp();
+        }
+        __syncthreads();
+        if (staged) {
+            const int ne = E * n_tiles;
+            for (int q = tid; q < ne; q += kLThreads) tile_base[q] = mat[q];
+        }
     }
-    for (int q = tid; q < R * R; q += kBlock) acc_splits[q] = 0;
+
+    // ------------------------------------ phase 3: offsets and splits ---
+    if (tid < E) ctot[tid] = ((ctot[tid] + align - 1) / align) * align;
     __syncthreads();
-    const int total = block_exclusive_scan<MOE_MAX_E / kBlock>(padded, E, scratch);
-    for (int q = tid; q < E; q += kBlock) offsets[q] = padded[q];
+    const int total = block_exclusive_scan_1024(ctot, E, scratch);
+    if (tid < E) offsets[tid] = ctot[tid];
     if (tid == 0) offsets[E] = total;
-
-    // splits[s][r] = sum over el of counts[s][r][el]; counts is [R*R][El]
-    // contiguous: load a batch of elements per thread (coalesced), then add
-    // each to its (s, r) bin in shared memory.
-    const int n = R * E;
-    constexpr int kSplitBatch = 8;
-    for (int base = 0; base < n; base += kBlock * kSplitBatch) {
-        int v[kSplitBatch];
-#pragma unroll
-        for (int b = 0; b < kSplitBatch; ++b) {
-            const int i = base + b * kBlock + tid;
-            v[b] = (i < n) ? __ldcg(counts + i) : 0;
-        }
-#pragma unroll
-        for (int b = 0; b < kSplitBatch; ++b) {
-            const int i = base + b * kBlock + tid;
-            if (i < n && v[b]) atomicAdd(&acc_splits[i / El], v[b]);
-        }
-    }
-    __syncthreads();
-    for (int q = tid; q < R * R; q += kBlock) splits[q] = acc_splits[q];
-    if (tid == 0) hdr->done = 0u;
+    for (int q = tid; q < R * R; q += kLThreads) splits[q] = acc_splits[q];
 }
 
 cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int align,
@@ -243,22 +341,54 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
     char* ws = static_cast<char*>(workspace);
 
     const int na_max = geo.TT * K;
-    const size_t hist_smem = sizeof(unsigned long long) * geo.TT + sizeof(int) * na_max +
-                             sizeof(uint16_t) * ((na_max + 1) & ~1) +
-                             sizeof(uint16_t) * (size_t)((na_max + 31) / 32) * E;
-    const int hist_grid = geo.n_tiles > 0 ? geo.n_tiles : 1;
-    layout_hist_kernel<<<hist_grid, kBlock, hist_smem, stream>>>(topk_idx, T, K, E, R, geo,
-                                                                 is_token_in_rank, ws, wl, status);
-    cudaError_t err = cudaGetLastError();
+    const size_t p1 = sizeof(unsigned long long) * geo.TT + sizeof(int) * na_max +
+                      sizeof(uint16_t) * ((na_max + 1) & ~1) +
+                      sizeof(uint16_t) * (size_t)((na_max + 31) / 32) * E;
+    const size_t p2 = sizeof(int) * ((size_t)kLWarps * (R + 1) + E + (size_t)R * R);
+    const size_t stage = sizeof(int) * (size_t)(E + R) * geo.n_tiles;
+    const int staged = (p2 + stage) <= kLayoutSmemMax ? 1 : 0;
+    const size_t p2s = p2 + (staged ? stage : 0);
+    const size_t smem = p1 > p2s ? p1 : p2s;
+    static int configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    if (smem > 48 * 1024 && dev >= 0 && dev < 64 && configured[dev] < (int)smem) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured[dev] = (int)smem;
+    }
+    // Zero the arrival counter, then one launch: cooperative (grid barriers)
+    // when one CTA per tile fits on the GPU at once, else last-CTA.
+    LayoutHeader* hdr = reinterpret_cast<LayoutHeader*>(ws);
+    cudaError_t err = cudaMemsetAsync(&hdr->done, 0, sizeof(hdr->done), stream);
     if (err != cudaSuccess) return err;
-
-    const int scan_grid = (E + R + kWarps - 1) / kWarps;
-    size_t scan_smem = sizeof(int) * (size_t)kWarps * (R + 1);
-    const size_t last_smem = sizeof(int) * ((size_t)E + (size_t)R * R);
-    if (scan_smem < last_smem) scan_smem = last_smem;
-    layout_scan_kernel<<<scan_grid, kBlock, scan_smem, stream>>>(
-        E, R, align, geo, tokens_per_expert, counts, splits, tokens_per_rank, expert_offsets, ws,
-        wl);
+    const int grid = geo.n_tiles > 0 ? geo.n_tiles : 1;
+    int coop = grid <= sm_count_current_device() ? 1 : 0;
+    if (coop) {
+        static int coop_ok[64] = {};
+        if (dev >= 0 && dev < 64 && coop_ok[dev] == 0) {
+            int attr = 0;
+            cudaDeviceGetAttribute(&attr, cudaDevAttrCooperativeLaunch, dev);
+            coop_ok[dev] = attr ? 1 : -1;
+        }
+        if (dev < 0 || dev >= 64 || coop_ok[dev] != 1) coop = 0;
+    }
+    // With barriers, phase 2 reads the rows from global memory: no staging.
+    const int stg = coop ? 0 : staged;
+    if (coop) {
+        void* args[] = {(void*)&topk_idx, (void*)&T, (void*)&K, (void*)&E, (void*)&R,
+                        (void*)&align, (void*)&geo, (void*)&tokens_per_expert, (void*)&counts,
+                        (void*)&splits, (void*)&tokens_per_rank, (void*)&is_token_in_rank,
+                        (void*)&expert_offsets, (void*)&ws, (void*)&wl, (void*)&status,
+                        (void*)&coop, (void*)&stg};
+        return cudaLaunchCooperativeKernel((const void*)layout_kernel, dim3(grid), dim3(kLThreads),
+                                           args, smem, stream);
+    }
+    layout_kernel<<<grid, kLThreads, smem, stream>>>(topk_idx, T, K, E, R, align, geo,
+                                                     tokens_per_expert, counts, splits,
+                                                     tokens_per_rank, is_token_in_rank,
+                                                     expert_offsets, ws, wl, status, coop, stg);
     return cudaGetLastError();
 }
 

@@ -85,6 +85,8 @@ extern "C" {
 #define MOE_ST_ROW_OOR 4          /* a flat_to_row entry outside [0, N_cap)     */
 #define MOE_ST_COVERAGE 8         /* row maps do not cover each (token, slot) once */
 #define MOE_ST_LAYOUT_MISMATCH 16 /* workspace was built for another (T, K, E)  */
+#define MOE_ST_TIMEOUT 32         /* a bounded grid barrier gave up (outputs
+                                     undefined; the kernel returned)         */
 
 /* Routing-weight ("router") dtypes. */
 #define MOE_DTYPE_F32 0

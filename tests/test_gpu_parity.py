@@ -70,7 +70,9 @@ def test_tiny_twice_deterministic():
     (64, 32, 64, 32, 2, 2),      # K=32 (maximum)
     (256, 16, 1024, 4, 64, 1),   # E=1024 and R=64 (maxima)
     (130, 8192, 8, 2, 2, 16),    # wide rows
-    (66, 8200, 4, 2, 2, 8),      # rows longer than one stand-in stage (cut into pieces)
+    (66, 8200, 4, 2, 2, 8),      # long rows
+    (20000, 8, 64, 8, 1, 4),     # more layout tiles than SMs: last-CTA path, staged
+    (4864, 8, 1024, 32, 8, 1),   # more tiles than SMs, count matrix too big to stage
 ])
 def test_edge_shapes(T, H, E, K, R, align):
     inp = custom_inputs(T, H, E, K, seed=T * 7 + K)

@@ -4,8 +4,8 @@ backward, on synthetic seeded inputs resident in HBM.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload qwen3|dsv3|dsv3_skew|mixtral|tiny]
 
-Step (eight kernels, all through the C ABI of libmoe_dispatch.so):
-  layout (2 kernels) -> permute -> stand-in experts -> weighted combine
+Step (seven kernels, all through the C ABI of libmoe_dispatch.so):
+  layout -> permute -> stand-in experts -> weighted combine
   -> combine backward -> stand-in backward -> unit-weight combine.
 
 Default workload: Qwen3-MoE-shaped fwd+bwd (T=16384 tokens, H=2048, E=128 in
@@ -43,13 +43,13 @@ METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak), 1 GP
 FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
 
-# Step names -> the kernel function each launches (combine_tma_kernel when the
-# gathered rows exceed L2, combine_kernel otherwise).
+# Step names -> the kernel function each launches (for K <= 8; larger K uses
+# the generic combine_kernel / combine_bwd_kernel).
 KERNEL_FUNCTION = {
-    "layout": "layout_hist_kernel+layout_scan_kernel", "permute": "permute_kernel",
+    "layout": "layout_kernel", "permute": "permute_kernel",
     "expert_scale": "expert_scale_kernel", "expert_scale_bwd": "expert_scale_kernel",
-    "combine": "combine_kernel", "dispatch_backward": "combine_kernel",
-    "combine_backward": "combine_bwd_kernel",
+    "combine": "combine_slots_kernel", "dispatch_backward": "combine_slots_kernel",
+    "combine_backward": "combine_bwd_slots_kernel",
 }
 
 KERNEL_SOURCES = {
@@ -205,7 +205,7 @@ class Path:
 
     names = ["layout", "permute", "expert_scale", "combine", "combine_backward", "expert_scale_bwd",
              "dispatch_backward"]
-    kernels_per_step = 8   # layout is two kernels
+    kernels_per_step = 7   # layout, permute, 2x expert_scale, 2x combine, combine backward
 
     def step(self, events=None):
         api, c = self.api, self.cfg

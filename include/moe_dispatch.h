@@ -37,8 +37,9 @@
  * --------------------------------
  *  - Every data pointer is caller-owned DEVICE memory of the current device.
  *    The library allocates nothing and never synchronises with the host;
- *    every call only enqueues kernels on `stream` (a cudaStream_t; NULL is
- *    the legacy default stream) and returns.  Results are defined once the
+ *    every call only enqueues work on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and returns: kernels, plus for the layout a
+ *    4-byte memset of its workspace counter.  Results are defined once the
  *    stream reaches them.  The only state kept between calls is a per-device
  *    cache of the SM count.
  *  - Notation: T tokens, H hidden size (bf16 elements per row), E experts,
@@ -133,7 +134,12 @@ int64_t moe_worst_case_rows(int T, int K, int E, int align);
  *                                     takes no rows)
  *      workspace                      moe_layout_workspace_bytes(T,K,E,R)
  *                                     bytes, 16-byte aligned
- * Status: MOE_ST_EXPERT_OOR (that assignment is left out of every count).
+ * Launch: one kernel of about one 1024-thread CTA per SM, cooperative (its
+ * phases are separated by grid barriers) when all its CTAs fit on the GPU at
+ * once; a barrier that does not complete within 2 s gives up and sets
+ * MOE_ST_TIMEOUT.
+ * Status: MOE_ST_EXPERT_OOR (that assignment is left out of every count),
+ *         MOE_ST_TIMEOUT.
  * Errors: MOE_ERR_INVALID_ARG for a null pointer, sizes outside the limits,
  *         align < 1, misalignment. */
 int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int align,

@@ -299,8 +299,12 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
 // order with D row chunks of y in flight (a ring): the dot product with g
 // accumulates in fp64 per slot (registers, across chunks), and the slot's
 // gradient chunk bf16_rn(w_k * g) is stored as a contiguous run.
+#ifndef MOE_BWD_MIN_BLOCKS
+#define MOE_BWD_MIN_BLOCKS 2
+#endif
+
 template <int KT, int U, int D>
-__global__ void __launch_bounds__(kBlock)
+__global__ void __launch_bounds__(kBlock, MOE_BWD_MIN_BLOCKS)
 combine_bwd_slots_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ rows,
                          int64_t N_cap, const int32_t* __restrict__ r2f,
                          const int32_t* __restrict__ f2r, const void* __restrict__ w, int wdtype,
@@ -428,8 +432,11 @@ static void launch_combine_t(int K, int grid, cudaStream_t st, const uint16_t* r
 
 // Enough warps for one token each (up to 8 resident CTAs per SM), and, when a
 // row sweep follows, enough threads to cover the rows.
-static int grid_tokens_and_rows(int T, int64_t N_cap, bool sweep_rows) {
-    const int cap = sm_count_current_device() * 8;
+#ifndef MOE_BWD_GRID_PER_SM
+#define MOE_BWD_GRID_PER_SM 8
+#endif
+static int grid_tokens_and_rows(int T, int64_t N_cap, bool sweep_rows, int per_sm = 8) {
+    const int cap = sm_count_current_device() * per_sm;
     int64_t want = (T + kWarps - 1) / kWarps;
     if (sweep_rows) {
         const int64_t rw = (N_cap + kBlock - 1) / kBlock;
@@ -466,7 +473,10 @@ cudaError_t launch_combine(const uint16_t* rows, int64_t N_cap, const int32_t* r
         const int u = K == 1 ? 4 * MOE_COMBINE_U : (K == 2 ? 2 * MOE_COMBINE_U : MOE_COMBINE_U);
         const int chunks = (n16 + 32 * u - 1) / (32 * u);
         const int64_t items = (int64_t)T * chunks;
-        const int cap = sm_count_current_device() * 8;
+#ifndef MOE_COMBINE_GRID_PER_SM
+#define MOE_COMBINE_GRID_PER_SM 8
+#endif
+        const int cap = sm_count_current_device() * MOE_COMBINE_GRID_PER_SM;
         int64_t want = (items + kWarps - 1) / kWarps;
         if (validate) {
             const int64_t rw = (N_cap + kBlock - 1) / kBlock;
@@ -505,7 +515,7 @@ cudaError_t launch_combine_backward(const uint16_t* grad_out, const uint16_t* ro
                                     const int32_t* expert_offsets, int E, int zero_pad,
                                     uint16_t* grad_rows, void* grad_weights, int32_t* status,
                                     cudaStream_t stream) {
-    const int grid = grid_tokens_and_rows(T, N_cap, zero_pad != 0);
+    const int grid = grid_tokens_and_rows(T, N_cap, zero_pad != 0, MOE_BWD_GRID_PER_SM);
     constexpr int U = MOE_COMBINE_U, D = MOE_COMBINE_D;
     switch (K) {
         case 1: combine_bwd_slots_kernel<1, 4 * U, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;

@@ -11,6 +11,13 @@
 
 namespace moe {
 
+#ifndef MOE_SCALE_U
+#define MOE_SCALE_U 4
+#endif
+#ifndef MOE_SCALE_GRID_PER_SM
+#define MOE_SCALE_GRID_PER_SM 64
+#endif
+
 template <int U>
 __global__ void __launch_bounds__(kBlock)
 expert_scale_kernel(const uint16_t* __restrict__ rows, int64_t N_cap,
@@ -71,11 +78,11 @@ cudaError_t launch_expert_scale(const uint16_t* rows, int64_t N_cap, const int32
                                 cudaStream_t stream) {
     const int sms = sm_count_current_device();
     int64_t want = (N_cap + kWarps - 1) / kWarps;
-    int grid = sms * 8;
+    int grid = sms * MOE_SCALE_GRID_PER_SM;
     if (want < grid) grid = (int)want;
     if (grid < 1) grid = 1;
     const size_t smem = sizeof(int) * (2 * (size_t)E + 1) + sizeof(float) * (size_t)E;
-    expert_scale_kernel<4><<<grid, kBlock, smem, stream>>>(rows, N_cap, expert_offsets,
+    expert_scale_kernel<MOE_SCALE_U><<<grid, kBlock, smem, stream>>>(rows, N_cap, expert_offsets,
                                                            tokens_per_expert, E, H, scales, out,
                                                            status);
     return cudaGetLastError();

@@ -304,7 +304,7 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
                                       staged ? mat + (size_t)p * n_tiles : nullptr, bs, counts,
                                       tokens_per_rank);
             if (p < E) {
-                const int r = p / El, el = p - r * El;
+                const int r = p / El;
                 for (int sb = lane; sb < R; sb += 32)
                     atomicAdd(&acc_splits[sb * R + r], bs[sb + 1] - bs[sb]);
                 if (lane == 0) {

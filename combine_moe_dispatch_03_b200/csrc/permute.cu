@@ -130,13 +130,19 @@ cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, in
                            int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
     // Enough CTAs to fill every SM several times over; the kernel strides
     // over its uniform items (token pieces, then pad-row pieces <= N_cap - A).
-    constexpr int U = 8;
+#ifndef MOE_PERMUTE_U
+#define MOE_PERMUTE_U 8
+#endif
+    constexpr int U = MOE_PERMUTE_U;
     const int sms = sm_count_current_device();
     const int n16 = H >> 3;
     const int64_t pieces = (n16 + 32 * U - 1) / (32 * U);
     const int64_t items = ((int64_t)T + (N_cap - (int64_t)T * K)) * pieces;
     int64_t grid = (items + kWarps - 1) / kWarps;
-    if (grid > (int64_t)sms * 8) grid = (int64_t)sms * 8;
+#ifndef MOE_PERMUTE_GRID_PER_SM
+#define MOE_PERMUTE_GRID_PER_SM 32
+#endif
+    if (grid > (int64_t)sms * MOE_PERMUTE_GRID_PER_SM) grid = (int64_t)sms * MOE_PERMUTE_GRID_PER_SM;
     if (grid < 1) grid = 1;
     permute_kernel<U><<<(int)grid, kBlock, sizeof(int) * 2 * ((size_t)E + 1), stream>>>(
         x, topk_idx, T, K, E, H, expert_offsets, static_cast<const char*>(workspace), zero_pad,

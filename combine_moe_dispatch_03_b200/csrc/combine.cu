@@ -516,7 +516,13 @@ cudaError_t launch_combine_backward(const uint16_t* grad_out, const uint16_t* ro
                                     uint16_t* grad_rows, void* grad_weights, int32_t* status,
                                     cudaStream_t stream) {
     const int grid = grid_tokens_and_rows(T, N_cap, zero_pad != 0, MOE_BWD_GRID_PER_SM);
-    constexpr int U = MOE_COMBINE_U, D = MOE_COMBINE_D;
+#ifndef MOE_BWD_U
+#define MOE_BWD_U MOE_COMBINE_U
+#endif
+#ifndef MOE_BWD_D
+#define MOE_BWD_D MOE_COMBINE_D
+#endif
+    constexpr int U = MOE_BWD_U, D = MOE_BWD_D;
     switch (K) {
         case 1: combine_bwd_slots_kernel<1, 4 * U, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
         case 2: combine_bwd_slots_kernel<2, 2 * U, 2><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;

@@ -217,3 +217,16 @@ def combine_backward(grad_out: torch.Tensor, rows: torch.Tensor, row_to_flat: to
                                     _ptr(grad_rows), _ptr(grad_w), _ptr(st), _stream(rows.device))
     check_rc(rc, "moe_combine_backward")
     return grad_rows, grad_w
+
+
+def scatter_flat_index(row_flat: torch.Tensor, T: int, K: int,
+                       status: torch.Tensor | None = None, out: torch.Tensor | None = None):
+    """flat_to_row [T,K] from the flat index each gathered row holds (-1: none),
+    with the folded restore's coverage check (MOE_ST_COVERAGE)."""
+    _require(row_flat, "row_flat", torch.int32, 1)
+    f2r = out if out is not None else torch.empty(T, K, dtype=torch.int32, device=row_flat.device)
+    st = status if status is not None else new_status(row_flat.device)
+    rc = lib().moe_scatter_flat_index(_ptr(row_flat), row_flat.shape[0], T, K, _ptr(f2r),
+                                      _ptr(st), _stream(row_flat.device))
+    check_rc(rc, "moe_scatter_flat_index")
+    return f2r

@@ -161,6 +161,16 @@ int moe_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t
                                                zero_pad, grad_rows, grad_weights, status, stream));
 }
 
+int moe_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
+                           int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
+    if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || N < 0 || N > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (!status || (N > 0 && !row_flat) || (T > 0 && !flat_to_row)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(row_flat, 4) || !aligned(flat_to_row, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    return finish(moe::launch_scatter_flat_index(row_flat, N, T, K, flat_to_row, status, stream));
+}
+
 const char* moe_strerror(int code) {
     switch (code) {
         case MOE_OK: return "ok";

@@ -239,6 +239,24 @@ int moe_combine_weighted(const uint16_t* rows, int64_t N_cap, const int32_t* row
                          int T, int K, int H, int validate, uint16_t* out, int32_t* status,
                          cudaStream_t stream);
 
+/* Scatter step of the folded restore ([DS-8847] Change: the rows of all
+ * tensor-parallel peers are gathered together with ONE flat index per row,
+ * token * top_k + slot; the routing data is scattered into [tokens, top_k];
+ * a clear RuntimeError is raised if the gathered rows do not cover every
+ * (token, slot)).  Builds the map moe_combine_weighted needs from the
+ * gathered rows' flat indices:
+ *
+ *   flat_to_row[f] = the row r with row_flat[r] == f
+ *
+ * In:  row_flat [N] int32 -- the flat index each gathered row holds, -1 for a
+ *      row holding none (a pad row).
+ * Out: flat_to_row [T,K] int32.
+ * Status: MOE_ST_COVERAGE if some f in [0, T*K) is held by no row or by more
+ *         than one, or a row holds an index outside [-1, T*K); flat_to_row is
+ *         then undefined.  Enqueues a memset and two small kernels. */
+int moe_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
+                           int32_t* flat_to_row, int32_t* status, cudaStream_t stream);
+
 /* Backward of fused_weighted_restore ([DS-8847] Tests: row and score
  * gradients; Benchmark: score gradient in FP32; [DeepEP-272]: the backward
  * of combine is a dispatch).  With g = grad_out [T,H]:

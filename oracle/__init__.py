@@ -72,6 +72,8 @@ def _load():
         lib.oracle_combine.restype = I
         lib.oracle_check_coverage.argtypes = [P, P, L, L]
         lib.oracle_check_coverage.restype = I
+        lib.oracle_scatter_flat_index.argtypes = [P, L, L, P]
+        lib.oracle_scatter_flat_index.restype = I
         lib.oracle_combine_backward.argtypes = [P, P, L, P, P, P, I, I, I, P, I, I, P, P]
         lib.oracle_combine_backward.restype = I
         _lib = lib
@@ -207,6 +209,15 @@ def check_coverage(row_to_flat: np.ndarray, flat_to_row: np.ndarray) -> int:
     flat_to_row = _c(flat_to_row, np.int32)
     return _load().oracle_check_coverage(_p(row_to_flat), _p(flat_to_row), row_to_flat.shape[0],
                                          flat_to_row.size)
+
+
+def scatter_flat_index(row_flat: np.ndarray, T: int, K: int) -> dict:
+    """flat_to_row [T,K] from the flat index each gathered row holds, with
+    the coverage check of the folded restore."""
+    row_flat = _c(row_flat, np.int32)
+    f2r = np.empty((T, K), np.int32)
+    st = _load().oracle_scatter_flat_index(_p(row_flat), row_flat.shape[0], T * K, _p(f2r))
+    return dict(flat_to_row=f2r, status=st)
 
 
 def combine_backward(grad_out_bf16: np.ndarray, rows_bf16: np.ndarray, row_to_flat: np.ndarray,

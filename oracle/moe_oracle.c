@@ -348,6 +348,35 @@ int oracle_check_coverage(const int32_t* row_to_flat, const int32_t* flat_to_row
     return 0;
 }
 
+/* Folded restore, scatter step [DS-8847] (Change: "all-gathers one flat
+ * index (token * top_k + slot) ... scatters them into [tokens, top_k]" and
+ * "raises a clear RuntimeError if the gathered rows do not cover every
+ * (token, slot)"): given the flat index held by each gathered row (-1 for a
+ * row holding none), flat_to_row[f] = the row holding f.  Every f in [0, A)
+ * must be held by exactly one row; a missing f, an f held twice, or an index
+ * outside [-1, A) returns ORC_COVERAGE (flat_to_row is then -1 where no row,
+ * or the first row, holds f). */
+int oracle_scatter_flat_index(const int32_t* row_flat, int64_t N, int64_t A, int32_t* flat_to_row) {
+    int status = 0;
+    for (int64_t f = 0; f < A; ++f) flat_to_row[f] = -1;
+    for (int64_t row = 0; row < N; ++row) {
+        int64_t f = row_flat[row];
+        if (f == -1) continue;
+        if (f < 0 || f >= A) {
+            status |= ORC_COVERAGE;
+            continue;
+        }
+        if (flat_to_row[f] >= 0) {
+            status |= ORC_COVERAGE;
+            continue;
+        }
+        flat_to_row[f] = (int32_t)row;
+    }
+    for (int64_t f = 0; f < A; ++f)
+        if (flat_to_row[f] < 0) status |= ORC_COVERAGE;
+    return status;
+}
+
 /* ---------------------------------------------------- combine backward --- */
 
 /* The backward of fused_weighted_restore [DS-8847] (Tests: "row and score

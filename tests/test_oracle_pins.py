@@ -500,3 +500,35 @@ def test_error_scale_matches_pages(orc):
                               w, lay["expert_offsets"])
     gw32 = bw["grad_w"].astype(np.float32)
     assert rel_l2(gw32, bw["grad_w"]) <= max(r[2] for r in table)
+
+
+# --------------------------------------------- folded restore: the scatter ---
+
+def test_scatter_flat_index_inverts_the_permute(orc):
+    """Scattering the flat index of every row (row_to_flat, as the gathered
+    metadata) reproduces flat_to_row exactly -- the two maps are inverses
+    ([DS-8847] Change: the flat index is scattered into [tokens, top_k])."""
+    inp, cfg, lay, pm, y = _tiny_pipeline(orc)
+    sc = orc.scatter_flat_index(pm["row_to_flat"], cfg.T, cfg.K)
+    assert sc["status"] == 0
+    np.testing.assert_array_equal(sc["flat_to_row"], pm["flat_to_row"])
+    # any order of the gathered rows: scattering a shuffled copy gives the
+    # shuffled positions
+    perm = np.random.default_rng(2).permutation(pm["row_to_flat"].shape[0])
+    sc2 = orc.scatter_flat_index(pm["row_to_flat"][perm], cfg.T, cfg.K)
+    assert sc2["status"] == 0
+    np.testing.assert_array_equal(perm[sc2["flat_to_row"]], pm["flat_to_row"])
+
+
+def test_scatter_flat_index_rejects_bad_coverage(orc):
+    """[DS-8847] Tests: a missing (token, slot) raises instead of reading an
+    unset row; also a duplicated and an out-of-range flat index."""
+    row_flat = np.array([3, 0, -1, 2, 1, 5, 4, -1], np.int32)   # T=3, K=2
+    assert orc.scatter_flat_index(row_flat, 3, 2)["status"] == 0
+    missing = row_flat.copy(); missing[5] = -1
+    r = orc.scatter_flat_index(missing, 3, 2)
+    assert r["status"] == orc.COVERAGE and r["flat_to_row"][2, 1] == -1
+    dup = row_flat.copy(); dup[2] = 3
+    assert orc.scatter_flat_index(dup, 3, 2)["status"] == orc.COVERAGE
+    bad = row_flat.copy(); bad[7] = 6
+    assert orc.scatter_flat_index(bad, 3, 2)["status"] == orc.COVERAGE

@@ -76,6 +76,12 @@ def _load():
         lib.oracle_scatter_flat_index.restype = I
         lib.oracle_combine_backward.argtypes = [P, P, L, P, P, P, I, I, I, P, I, I, P, P]
         lib.oracle_combine_backward.restype = I
+        lib.oracle_permute_payload.argtypes = [P, L, P, L, P, I, I, I, P, I, L, P, P, P, P]
+        lib.oracle_permute_payload.restype = I
+        lib.oracle_combine_f32.argtypes = [P, L, P, P, I, I, I, P, P]
+        lib.oracle_combine_f32.restype = I
+        lib.oracle_combine_backward_f32.argtypes = [P, P, L, P, P, P, I, I, I, P, I, I, P, P]
+        lib.oracle_combine_backward_f32.restype = I
         _lib = lib
         return lib
 
@@ -243,3 +249,76 @@ def combine_backward(grad_out_bf16: np.ndarray, rows_bf16: np.ndarray, row_to_fl
                                          _p(flat_to_row), _p(w), T, K, H, _p(expert_offsets), E,
                                          int(bool(zero_pad)), _p(grad_rows), _p(grad_w))
     return dict(grad_rows=grad_rows, grad_w=grad_w, status=st)
+
+
+# ----------------------------------------------- payload and fp32 variants ---
+
+def permute_payload(x: np.ndarray, topk_idx: np.ndarray, E: int, expert_offsets: np.ndarray,
+                    N_cap: int, aux: np.ndarray | None = None, zero_pad: bool = True,
+                    x_perm_init: np.ndarray | None = None,
+                    aux_perm_init: np.ndarray | None = None) -> dict:
+    """Dispatch of opaque row payloads: x [T, ...] (any dtype, each token row
+    row_bytes bytes) and optionally aux [T, ...] (e.g. FP8 scales)."""
+    x = np.ascontiguousarray(x)
+    topk_idx = _c(topk_idx, np.int64)
+    expert_offsets = _c(expert_offsets, np.int32)
+    T = x.shape[0]
+    K = topk_idx.shape[1]
+    row_bytes = x.nbytes // T if T else x.dtype.itemsize * int(np.prod(x.shape[1:]))
+    shape = (N_cap,) + x.shape[1:]
+    xp = (np.zeros(shape, x.dtype) if x_perm_init is None
+          else np.array(x_perm_init, dtype=x.dtype, copy=True, order="C"))
+    auxp, aux_bytes = None, 0
+    if aux is not None:
+        aux = np.ascontiguousarray(aux)
+        aux_bytes = aux.nbytes // T if T else aux.dtype.itemsize * int(np.prod(aux.shape[1:]))
+        ashape = (N_cap,) + aux.shape[1:]
+        auxp = (np.zeros(ashape, aux.dtype) if aux_perm_init is None
+                else np.array(aux_perm_init, dtype=aux.dtype, copy=True, order="C"))
+    r2f = np.empty(N_cap, np.int32)
+    f2r = np.empty((T, K), np.int32)
+    st = _load().oracle_permute_payload(_p(x), row_bytes, _p(aux), aux_bytes, _p(topk_idx), T, K, E,
+                                        _p(expert_offsets), int(bool(zero_pad)), N_cap, _p(xp),
+                                        _p(auxp), _p(r2f), _p(f2r))
+    return dict(x_perm=xp, aux_perm=auxp, row_to_flat=r2f, flat_to_row=f2r, status=st)
+
+
+def combine_f32(rows: np.ndarray, flat_to_row: np.ndarray, weights: np.ndarray | None,
+                seq: bool = True) -> dict:
+    """fused_weighted_restore on fp32 rows: fp64 reference and the FP32
+    fmaf-chain value (fp32 output)."""
+    rows = _c(rows, np.float32)
+    flat_to_row = _c(flat_to_row, np.int32)
+    T, K = flat_to_row.shape
+    N_cap, H = rows.shape
+    w = None if weights is None else _c(np.asarray(weights, np.float32), np.float32)
+    ref = np.empty((T, H), np.float64)
+    out_seq = np.empty((T, H), np.float32) if seq else None
+    st = _load().oracle_combine_f32(_p(rows), N_cap, _p(flat_to_row), _p(w), T, K, H, _p(ref),
+                                    _p(out_seq))
+    return dict(ref=ref, seq=out_seq, status=st)
+
+
+def combine_backward_f32(grad_out: np.ndarray, rows: np.ndarray, row_to_flat: np.ndarray,
+                         flat_to_row: np.ndarray, weights: np.ndarray, expert_offsets: np.ndarray,
+                         zero_pad: bool = True, grad_rows_init: np.ndarray | None = None,
+                         want_grad_w: bool = True) -> dict:
+    """Row gradients fp32(w*g) and fp64 weight gradients <g_t, y_row> for
+    fp32 rows."""
+    g = _c(grad_out, np.float32)
+    rows = _c(rows, np.float32)
+    row_to_flat = _c(row_to_flat, np.int32)
+    flat_to_row = _c(flat_to_row, np.int32)
+    expert_offsets = _c(expert_offsets, np.int32)
+    w = _c(np.asarray(weights, np.float32), np.float32)
+    T, K = flat_to_row.shape
+    N_cap, H = rows.shape
+    E = expert_offsets.shape[0] - 1
+    grad_rows = (np.zeros((N_cap, H), np.float32) if grad_rows_init is None
+                 else np.array(grad_rows_init, np.float32, copy=True, order="C"))
+    grad_w = np.empty((T, K), np.float64) if want_grad_w else None
+    st = _load().oracle_combine_backward_f32(_p(g), _p(rows), N_cap, _p(row_to_flat),
+                                             _p(flat_to_row), _p(w), T, K, H, _p(expert_offsets), E,
+                                             int(bool(zero_pad)), _p(grad_rows), _p(grad_w))
+    return dict(grad_rows=grad_rows, grad_w=grad_w, status=st)
+

@@ -240,6 +240,68 @@ int oracle_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int
     return status;
 }
 
+/* Dispatch of an arbitrary row payload ([DeepEP-272]: dispatch takes x as a
+ * bf16 tensor or as an FP8 tuple (data, scales); [DS-8847] Tests: fp32 and
+ * bf16 rows).  The rows are opaque bytes: every token row of x is row_bytes
+ * bytes and, when aux != NULL, every token also owns an aux row of aux_bytes
+ * bytes (the FP8 scales), which travels with it.  The destination row of
+ * each assignment is the one oracle_permute defines -- the i-th assignment
+ * of expert e in (expert, flat index) order lands on offsets[e] + i -- found
+ * here with the same sort:
+ *
+ *   x_perm[row(f)] = x[t]     aux_perm[row(f)] = aux[t]
+ *   maps, pad rows (zero, both payloads, when zero_pad) and the untouched
+ *   tail exactly as in oracle_permute. */
+int oracle_permute_payload(const uint8_t* x, int64_t row_bytes, const uint8_t* aux,
+                           int64_t aux_bytes, const int64_t* topk_idx, int T, int K, int E,
+                           const int32_t* offsets, int zero_pad, int64_t N_cap, uint8_t* x_perm,
+                           uint8_t* aux_perm, int32_t* row_to_flat, int32_t* flat_to_row) {
+    int status = 0;
+    int64_t A = (int64_t)T * K;
+    orc_assign* list = (orc_assign*)malloc(sizeof(orc_assign) * (size_t)(A > 0 ? A : 1));
+    int64_t n = 0;
+    for (int64_t f = 0; f < A; ++f) {
+        flat_to_row[f] = -1;
+        int64_t e = topk_idx[f];
+        if (e < 0 || e >= E) {
+            status |= ORC_EXPERT_OOR;
+            continue;
+        }
+        list[n].expert = (int32_t)e;
+        list[n].flat = (int32_t)f;
+        ++n;
+    }
+    qsort(list, (size_t)n, sizeof(orc_assign), orc_cmp_assign);
+    for (int64_t row = 0; row < N_cap; ++row) row_to_flat[row] = -1;
+    if ((int64_t)offsets[E] > N_cap) status |= ORC_CAPACITY;
+
+    int64_t first = 0;   /* index in `list` of the current expert's first assignment */
+    for (int64_t i = 0; i < n; ++i) {
+        if (i == 0 || list[i].expert != list[i - 1].expert) first = i;
+        int32_t e = list[i].expert;
+        int64_t row = (int64_t)offsets[e] + (i - first);
+        int32_t f = list[i].flat;
+        if (row >= N_cap) {
+            status |= ORC_CAPACITY;
+            continue;
+        }
+        int64_t t = f / K;
+        memcpy(x_perm + row * row_bytes, x + t * row_bytes, (size_t)row_bytes);
+        if (aux) memcpy(aux_perm + row * aux_bytes, aux + t * aux_bytes, (size_t)aux_bytes);
+        row_to_flat[row] = f;
+        flat_to_row[f] = (int32_t)row;
+    }
+    if (zero_pad) {
+        for (int64_t row = 0; row < (int64_t)offsets[E] && row < N_cap; ++row)
+            if (row_to_flat[row] < 0) {
+                memset(x_perm + row * row_bytes, 0, (size_t)row_bytes);
+                if (aux) memset(aux_perm + row * aux_bytes, 0, (size_t)aux_bytes);
+            }
+    }
+    free(list);
+    return status;
+}
+
 /* The definition of the row written for assignment f, counted by brute force
  * in O(A^2): row(f) = offsets[e] + #{f' < f : topk_idx[f'] = e}.  Used only to
  * pin oracle_permute on small inputs. */
@@ -321,6 +383,38 @@ int oracle_combine(const uint16_t* rows, int64_t N_cap, const int32_t* flat_to_r
             }
             out_ref[(int64_t)t * H + h] = sum;
             if (out_seq) out_seq[(int64_t)t * H + h] = oracle_bf16_from_float(acc);
+        }
+    }
+    return status;
+}
+
+/* fused_weighted_restore on fp32 rows ([DS-8847] Tests: "fp32 and bf16
+ * rows"; the activation dtype is fp32, so the output is fp32 and the FP32
+ * accumulation is not followed by a narrower rounding).  out_ref receives
+ * the fp64 sum (a product of two floats is exact in fp64); out_seq, when not
+ * NULL, the FP32 reading: acc = 0, acc = fmaf(w, y, acc) for k = 0..K-1 in
+ * order, stored as is.  Out-of-range slots as in oracle_combine. */
+int oracle_combine_f32(const float* rows, int64_t N_cap, const int32_t* flat_to_row,
+                       const float* w, int T, int K, int H, double* out_ref, float* out_seq) {
+    int status = 0;
+    for (int t = 0; t < T; ++t) {
+        for (int h = 0; h < H; ++h) {
+            double sum = 0.0;
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                int64_t f = (int64_t)t * K + k;
+                int64_t row = flat_to_row[f];
+                if (row < 0 || row >= N_cap) {
+                    status |= ORC_ROW_OOR;
+                    continue;
+                }
+                float wk = w ? w[f] : 1.0f;
+                float y = rows[row * H + h];
+                sum += (double)wk * (double)y;
+                acc = fmaf(wk, y, acc);
+            }
+            out_ref[(int64_t)t * H + h] = sum;
+            if (out_seq) out_seq[(int64_t)t * H + h] = acc;
         }
     }
     return status;
@@ -415,6 +509,44 @@ int oracle_combine_backward(const uint16_t* g, const uint16_t* rows, int64_t N_c
     if (zero_pad) {
         for (int64_t row = 0; row < (int64_t)offsets[E] && row < N_cap; ++row)
             if (row_to_flat[row] < 0) memset(grad_rows + row * H, 0, sizeof(uint16_t) * (size_t)H);
+    }
+    return status;
+}
+
+/* Backward of the fp32-row restore ([DS-8847] Tests): with g = grad_out,
+ *
+ *   grad_rows[flat_to_row[f]] = fp32(w[f] * g[t])    (the product is exact in
+ *                                                     fp64, rounded once)
+ *   grad_w[f] = sum_h g[t,h] * rows[flat_to_row[f], h]           (fp64 sum)
+ *
+ * Pad rows and out-of-range slots as in oracle_combine_backward. */
+int oracle_combine_backward_f32(const float* g, const float* rows, int64_t N_cap,
+                                const int32_t* row_to_flat, const int32_t* flat_to_row,
+                                const float* w, int T, int K, int H, const int32_t* offsets,
+                                int E, int zero_pad, float* grad_rows, double* grad_w) {
+    int status = 0;
+    for (int t = 0; t < T; ++t)
+        for (int k = 0; k < K; ++k) {
+            int64_t f = (int64_t)t * K + k;
+            int64_t row = flat_to_row[f];
+            if (row < 0 || row >= N_cap) {
+                status |= ORC_ROW_OOR;
+                if (grad_w) grad_w[f] = 0.0;
+                continue;
+            }
+            double wk = (double)w[f];
+            double dot = 0.0;
+            for (int h = 0; h < H; ++h) {
+                double gv = (double)g[(int64_t)t * H + h];
+                double yv = (double)rows[row * H + h];
+                grad_rows[row * H + h] = (float)(wk * gv);
+                dot += gv * yv;
+            }
+            if (grad_w) grad_w[f] = dot;
+        }
+    if (zero_pad) {
+        for (int64_t row = 0; row < (int64_t)offsets[E] && row < N_cap; ++row)
+            if (row_to_flat[row] < 0) memset(grad_rows + row * H, 0, sizeof(float) * (size_t)H);
     }
     return status;
 }

@@ -532,3 +532,176 @@ def test_scatter_flat_index_rejects_bad_coverage(orc):
     assert orc.scatter_flat_index(dup, 3, 2)["status"] == orc.COVERAGE
     bad = row_flat.copy(); bad[7] = 6
     assert orc.scatter_flat_index(bad, 3, 2)["status"] == orc.COVERAGE
+
+
+# ------------------------------------------ payload dispatch, fp32 rows ---
+# [DeepEP-272]: dispatch takes x as bf16 or as an FP8 tuple (data, scales);
+# [DS-8847] Tests: the fused restore on fp32 and bf16 rows.
+
+def _routing_cases():
+    rng = np.random.default_rng(41)
+    cases = [(make_inputs("tiny")["topk_idx"].numpy(), 8, 8)]
+    for T, K, E, align in [(97, 5, 13, 4), (40, 3, 6, 1), (16, 2, 40, 3)]:
+        cases.append((rng.integers(0, E, size=(T, K)).astype(np.int64), E, align))  # repeats allowed
+    return cases
+
+
+def test_permute_payload_on_bf16_rows_equals_permute(orc):
+    """On bf16 rows (row_bytes = 2H, no aux) the payload dispatch is the
+    brute-force-pinned bf16 permute, bit for bit: rows, maps, pad zeros, the
+    untouched tail (pre-filled pattern), status -- with and without zero_pad."""
+    rng = np.random.default_rng(42)
+    for topk, E, align in _routing_cases():
+        T, K = topk.shape
+        lay = orc.layout(topk, E, 1, align)
+        off = lay["expert_offsets"]
+        N_cap = capacity_rows(T, K, E, align) + 3
+        x = rng.integers(0, 65535, size=(T, 24)).astype(np.uint16)
+        init = np.full((N_cap, 24), 0x4B4B, np.uint16)
+        for zp in (True, False):
+            a = orc.permute(x, topk, E, off, N_cap, zero_pad=zp, x_perm_init=init)
+            b = orc.permute_payload(x, topk, E, off, N_cap, zero_pad=zp, x_perm_init=init)
+            for key in ("x_perm", "row_to_flat", "flat_to_row", "status"):
+                np.testing.assert_array_equal(a[key], b[key])
+
+
+def test_permute_payload_rows_bruteforce_and_aux(orc):
+    """Every routing with T<=3, K<=2, E<=3: the rows are the definitional
+    count offsets[e] + #{f' < f : e(f') = e}; the aux row of token t lands on
+    every row of t, pad rows of both payloads are zero."""
+    n = 0
+    for T, K, E in [(2, 1, 3), (2, 2, 3), (3, 2, 2)]:
+        for align in (1, 3):
+            for topk in _all_routings(T, K, E):
+                lay = orc.layout(topk, E, 1, align)
+                off = lay["expert_offsets"]
+                N_cap = capacity_rows(T, K, E, align)
+                x = (np.arange(T * 16, dtype=np.uint8) + 1).reshape(T, 16)
+                aux = (np.arange(T * 3, dtype=np.float32) + 0.5).reshape(T, 3)
+                pm = orc.permute_payload(x, topk, E, off, N_cap, aux=aux)
+                f2r = pm["flat_to_row"]
+                np.testing.assert_array_equal(f2r, orc.bruteforce_rows(topk, E, off))
+                for f in range(T * K):
+                    np.testing.assert_array_equal(pm["x_perm"][f2r.flat[f]], x[f // K])
+                    np.testing.assert_array_equal(pm["aux_perm"][f2r.flat[f]], aux[f // K])
+                pad = np.flatnonzero(pm["row_to_flat"][: off[-1]] < 0)
+                assert not pm["x_perm"][pad].any() and not pm["aux_perm"][pad].any()
+                n += 1
+    assert n > 200
+
+
+def test_permute_payload_fp8_tuple_dequantizes_to_the_token(orc):
+    """An FP8 (data, scales) payload -- e4m3 data with one fp32 scale per 128
+    columns, quantised with torch -- arrives on every row of its token byte
+    for byte, so every dispatched row dequantises to its token's values."""
+    inp = make_inputs("tiny")
+    cfg = inp["cfg"]
+    x = inp["x"].float()
+    blocks = x.view(cfg.T, cfg.H // 128, 128)
+    scales = (blocks.abs().amax(-1) / 448.0).clamp_min(1e-12)
+    data = (blocks / scales[..., None]).to(torch.float8_e4m3fn).view(cfg.T, cfg.H)
+    d8 = data.view(torch.uint8).numpy()
+    topk = inp["topk_idx"].numpy()
+    lay = orc.layout(topk, cfg.E, cfg.R, cfg.align)
+    N_cap = capacity_rows(cfg.T, cfg.K, cfg.E, cfg.align)
+    pm = orc.permute_payload(d8, topk, cfg.E, lay["expert_offsets"], N_cap,
+                             aux=scales.numpy().astype(np.float32))
+    deq_tok = (data.float().view(cfg.T, -1, 128) * scales[..., None]).view(cfg.T, cfg.H).numpy()
+    rows = torch.from_numpy(pm["x_perm"]).view(torch.float8_e4m3fn).float()
+    sc = torch.from_numpy(pm["aux_perm"])
+    deq_rows = (rows.view(N_cap, -1, 128) * sc[..., None]).view(N_cap, cfg.H).numpy()
+    f2r = pm["flat_to_row"]
+    for t in range(cfg.T):
+        for k in range(cfg.K):
+            np.testing.assert_array_equal(deq_rows[f2r[t, k]], deq_tok[t])
+
+
+def test_combine_f32_on_bf16_values_is_the_bf16_combine(orc):
+    """fp32 rows holding bf16 values: the fp64 reference is the bf16
+    combine's, exactly, and the FP32 chain rounded once to bf16 is the bf16
+    combine's FP32 result (both pinned by the round trip, the adjoint and the
+    page's error scale)."""
+    inp, cfg, lay, pm, y = _tiny_pipeline(orc)
+    w = inp["weights"].numpy()
+    a = orc.combine(y, pm["flat_to_row"], w)
+    b = orc.combine_f32(orc.f32_from_bf16(y), pm["flat_to_row"], w)
+    np.testing.assert_array_equal(a["ref"], b["ref"])
+    np.testing.assert_array_equal(a["seq"], orc.bf16_from_f32(b["seq"]))
+    c = orc.combine_f32(orc.f32_from_bf16(y), pm["flat_to_row"], None)
+    np.testing.assert_array_equal(orc.combine(y, pm["flat_to_row"], None)["ref"], c["ref"])
+
+
+def test_combine_f32_identity_and_error_bound(orc):
+    """K = 1, w = 1: the output is the row itself.  Random fp32 rows: the
+    FP32 chain is within the textbook bound of a K-term fmaf recursion,
+    |seq - ref| <= gamma_K * sum_k |w_k y_k|, gamma_K = K u / (1 - K u),
+    u = 2^-24."""
+    rng = np.random.default_rng(43)
+    T, K, H, N = 50, 1, 16, 80
+    rows = rng.standard_normal((N, H)).astype(np.float32)
+    f2r = rng.permutation(N)[:T].astype(np.int32).reshape(T, 1)
+    r = orc.combine_f32(rows, f2r, np.ones((T, 1), np.float32))
+    np.testing.assert_array_equal(r["seq"], rows[f2r[:, 0]])
+    T, K = 60, 8
+    f2r = rng.permutation(N + 400)[: T * K].astype(np.int32).reshape(T, K) % (N + 400)
+    rows = (rng.standard_normal((N + 400, H)) * 10.0 ** rng.integers(-3, 4, (N + 400, 1))).astype(np.float32)
+    w = rng.random((T, K)).astype(np.float32)
+    r = orc.combine_f32(rows, f2r, w)
+    mag = np.einsum("tk,tkh->th", np.abs(w).astype(np.float64), np.abs(rows[f2r]).astype(np.float64))
+    u = 2.0 ** -24
+    gamma = K * u / (1 - K * u)
+    assert (np.abs(r["seq"].astype(np.float64) - r["ref"]) <= gamma * mag).all()
+    assert (np.abs(r["seq"].astype(np.float64) - r["ref"]) > 0).any()
+
+
+def test_combine_backward_f32_on_bf16_values_is_the_bf16_backward(orc):
+    """bf16-valued fp32 inputs: the weight gradient is the bf16 backward's
+    (same fp64 sums, exactly) and the fp32 row gradient rounded once to bf16
+    is the bf16 backward's row gradient."""
+    inp, cfg, lay, pm, y = _tiny_pipeline(orc, with_grad=True)
+    w = inp["weights"].numpy()
+    g = bf16_bits(inp["grad_out"])
+    a = orc.combine_backward(g, y, pm["row_to_flat"], pm["flat_to_row"], w, lay["expert_offsets"])
+    b = orc.combine_backward_f32(orc.f32_from_bf16(g), orc.f32_from_bf16(y), pm["row_to_flat"],
+                                 pm["flat_to_row"], w, lay["expert_offsets"])
+    np.testing.assert_array_equal(a["grad_w"], b["grad_w"])
+    np.testing.assert_array_equal(a["grad_rows"], orc.bf16_from_f32(b["grad_rows"]))
+
+
+def test_combine_backward_f32_finite_differences(orc):
+    """Random fp32 rows: grad_w against central differences of the fp64
+    forward; grad_rows is fp32(w * g) (one rounding of the exact product)
+    against the adjoint <g, combine(y + dY)> - <g, combine(y)> = <grad_rows, dY>."""
+    rng = np.random.default_rng(44)
+    T, K, H, E = 24, 3, 32, 5
+    topk = rng.integers(0, E, size=(T, K)).astype(np.int64)
+    lay = orc.layout(topk, E, 1, 2)
+    N_cap = capacity_rows(T, K, E, 2)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    pm = orc.permute_payload(x, topk, E, lay["expert_offsets"], N_cap)
+    y = pm["x_perm"]
+    w = rng.random((T, K)).astype(np.float32)
+    g = rng.standard_normal((T, H)).astype(np.float32)
+    gd = g.astype(np.float64)
+    f2r, r2f = pm["flat_to_row"], pm["row_to_flat"]
+    bw = orc.combine_backward_f32(g, y, r2f, f2r, w, lay["expert_offsets"])
+    for (t, k) in [(0, 0), (3, 2), (11, 1), (23, 0)]:
+        wp = w.copy(); wm = w.copy()
+        wp[t, k] = np.float32(w[t, k] + np.float32(2 ** -6))
+        wm[t, k] = np.float32(w[t, k] - np.float32(2 ** -6))
+        hp = np.sum(gd * orc.combine_f32(y, f2r, wp, seq=False)["ref"])
+        hm = np.sum(gd * orc.combine_f32(y, f2r, wm, seq=False)["ref"])
+        fd = (hp - hm) / (float(wp[t, k]) - float(wm[t, k]))
+        assert abs(fd - bw["grad_w"][t, k]) <= 1e-9 * max(1.0, abs(fd))
+    dY = (rng.standard_normal(y.shape) * 0.01).astype(np.float32)
+    dY[r2f < 0] = 0
+    base = np.sum(gd * orc.combine_f32(y, f2r, w, seq=False)["ref"])
+    delta = np.sum(gd * orc.combine_f32(y + dY, f2r, w, seq=False)["ref"]) - base
+    dYeff = (y + dY).astype(np.float64) - y.astype(np.float64)
+    pred = np.sum(bw["grad_rows"].astype(np.float64) * dYeff)
+    assert abs(delta - pred) <= 2 ** -22 * np.sum(np.abs(bw["grad_rows"] * dYeff)) + 1e-12
+    real = f2r.reshape(-1)
+    tok = np.arange(T * K) // K
+    np.testing.assert_array_equal(bw["grad_rows"][real],
+                                  (w.reshape(-1, 1).astype(np.float64) * gd[tok]).astype(np.float32))
+    assert not bw["grad_rows"][: lay["expert_offsets"][-1]][r2f[: lay["expert_offsets"][-1]] < 0].any()

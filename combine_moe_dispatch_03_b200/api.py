@@ -16,6 +16,7 @@ Dispatch/Combine Support Autograd Like PyTorch's all_to_all?").
 from __future__ import annotations
 
 import dataclasses
+import math
 
 import torch
 
@@ -168,7 +169,10 @@ def combine_weighted(rows: torch.Tensor, flat_to_row: torch.Tensor,
                      validate: bool = False, status: torch.Tensor | None = None,
                      out: torch.Tensor | None = None):
     """fused_weighted_restore; weights=None is the unit-weight combine
-    (the backward of dispatch)."""
+    (the backward of dispatch).  bf16 rows give a bf16 output (FP32
+    accumulation, one rounding); fp32 rows an fp32 output."""
+    if isinstance(rows, torch.Tensor) and rows.dtype == torch.float32:
+        return _combine_weighted_f32(rows, flat_to_row, weights, row_to_flat, validate, status, out)
     _require(rows, "rows", torch.bfloat16, 2)
     _require(flat_to_row, "flat_to_row", torch.int32, 2)
     N_cap, H = rows.shape
@@ -196,7 +200,11 @@ def combine_backward(grad_out: torch.Tensor, rows: torch.Tensor, row_to_flat: to
                      flat_to_row: torch.Tensor, weights: torch.Tensor, layout: Layout,
                      zero_pad: bool = True, want_grad_weights: bool = True,
                      status: torch.Tensor | None = None, out: tuple | None = None):
-    """Returns (grad_rows [N_cap,H] bf16, grad_weights [T,K] router dtype or None)."""
+    """Returns (grad_rows [N_cap,H] in the rows' dtype (bf16 or fp32),
+    grad_weights [T,K] router dtype or None)."""
+    if isinstance(rows, torch.Tensor) and rows.dtype == torch.float32:
+        return _combine_backward_f32(grad_out, rows, row_to_flat, flat_to_row, weights, layout,
+                                     zero_pad, want_grad_weights, status, out)
     _require(grad_out, "grad_out", torch.bfloat16, 2)
     _require(rows, "rows", torch.bfloat16, 2)
     _require(flat_to_row, "flat_to_row", torch.int32, 2)
@@ -230,3 +238,89 @@ def scatter_flat_index(row_flat: torch.Tensor, T: int, K: int,
                                       _ptr(st), _stream(row_flat.device))
     check_rc(rc, "moe_scatter_flat_index")
     return f2r
+
+
+def _combine_weighted_f32(rows, flat_to_row, weights, row_to_flat, validate, status, out):
+    _require(rows, "rows", torch.float32, 2)
+    _require(flat_to_row, "flat_to_row", torch.int32, 2)
+    N_cap, H = rows.shape
+    T, K = flat_to_row.shape
+    wd = DTYPE_F32
+    if weights is not None:
+        wd = _weight_dtype(weights)
+        _require(weights, "weights", weights.dtype, 2)
+        if tuple(weights.shape) != (T, K):
+            raise ValueError("weights must be [T, K]")
+    if validate:
+        if row_to_flat is None:
+            raise ValueError("validate=True needs row_to_flat")
+        _require(row_to_flat, "row_to_flat", torch.int32, 1)
+    o = out if out is not None else torch.empty(T, H, dtype=torch.float32, device=rows.device)
+    st = status if status is not None else new_status(rows.device)
+    rc = lib().moe_combine_weighted_f32(_ptr(rows), N_cap, _ptr(row_to_flat), _ptr(flat_to_row),
+                                        _ptr(weights), wd, T, K, H, int(bool(validate)), _ptr(o),
+                                        _ptr(st), _stream(rows.device))
+    check_rc(rc, "moe_combine_weighted_f32")
+    return o
+
+
+def _combine_backward_f32(grad_out, rows, row_to_flat, flat_to_row, weights, layout, zero_pad,
+                          want_grad_weights, status, out):
+    _require(grad_out, "grad_out", torch.float32, 2)
+    _require(rows, "rows", torch.float32, 2)
+    _require(flat_to_row, "flat_to_row", torch.int32, 2)
+    _require(row_to_flat, "row_to_flat", torch.int32, 1)
+    wd = _weight_dtype(weights)
+    _require(weights, "weights", weights.dtype, 2)
+    N_cap, H = rows.shape
+    T, K = flat_to_row.shape
+    if out is None:
+        grad_rows = torch.empty_like(rows)
+        grad_w = torch.empty(T, K, dtype=weights.dtype, device=rows.device) if want_grad_weights else None
+    else:
+        grad_rows, grad_w = out
+    st = status if status is not None else new_status(rows.device)
+    rc = lib().moe_combine_backward_f32(_ptr(grad_out), _ptr(rows), N_cap, _ptr(row_to_flat),
+                                        _ptr(flat_to_row), _ptr(weights), wd, T, K, H,
+                                        _ptr(layout.expert_offsets), layout.E, int(bool(zero_pad)),
+                                        _ptr(grad_rows), _ptr(grad_w), _ptr(st), _stream(rows.device))
+    check_rc(rc, "moe_combine_backward_f32")
+    return grad_rows, grad_w
+
+
+def permute_payload(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout,
+                    aux: torch.Tensor | None = None, capacity: int | None = None,
+                    zero_pad: bool = True, status: torch.Tensor | None = None,
+                    out: tuple | None = None):
+    """Dispatch of an opaque row payload x [T, ...] (any dtype; e.g. the e4m3
+    data of an FP8 tuple, or fp32 rows) and an optional per-token aux payload
+    [T, ...] (e.g. the FP8 scales).  Returns (x_perm, aux_perm or None,
+    row_to_flat, flat_to_row)."""
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or not x.is_contiguous() or x.dim() < 1:
+        raise ValueError("x must be a contiguous CUDA tensor [T, ...]")
+    _require(topk_idx, "topk_idx", torch.int64, 2)
+    T = x.shape[0]
+    K = topk_idx.shape[1]
+    dev = x.device
+    row_bytes = x.element_size() * math.prod(x.shape[1:])
+    aux_bytes = 0
+    if aux is not None:
+        if not aux.is_cuda or not aux.is_contiguous() or aux.shape[0] != T:
+            raise ValueError("aux must be a contiguous CUDA tensor [T, ...]")
+        aux_bytes = aux.element_size() * math.prod(aux.shape[1:])
+    N_cap = capacity if capacity is not None else worst_case_rows(T, K, layout.E, layout.align)
+    if out is None:
+        x_perm = torch.empty((N_cap,) + tuple(x.shape[1:]), dtype=x.dtype, device=dev)
+        aux_perm = (torch.empty((N_cap,) + tuple(aux.shape[1:]), dtype=aux.dtype, device=dev)
+                    if aux is not None else None)
+        r2f = torch.empty(N_cap, dtype=torch.int32, device=dev)
+        f2r = torch.empty(T, K, dtype=torch.int32, device=dev)
+    else:
+        x_perm, aux_perm, r2f, f2r = out
+    st = status if status is not None else new_status(dev)
+    rc = lib().moe_permute_payload(_ptr(x), row_bytes, _ptr(aux), aux_bytes, _ptr(topk_idx), T, K,
+                                   layout.E, _ptr(layout.expert_offsets), _ptr(layout.workspace),
+                                   int(bool(zero_pad)), N_cap, _ptr(x_perm), _ptr(aux_perm),
+                                   _ptr(r2f), _ptr(f2r), _ptr(st), _stream(dev))
+    check_rc(rc, "moe_permute_payload")
+    return x_perm, aux_perm, r2f, f2r

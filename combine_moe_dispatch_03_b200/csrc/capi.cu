@@ -161,6 +161,74 @@ int moe_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t
                                                zero_pad, grad_rows, grad_weights, status, stream));
 }
 
+int moe_permute_payload(const void* x, int64_t row_bytes, const void* aux, int64_t aux_row_bytes,
+                        const int64_t* topk_idx, int T, int K, int E,
+                        const int32_t* expert_offsets, const void* workspace, int zero_pad,
+                        int64_t N_cap, void* x_perm, void* aux_perm, int32_t* row_to_flat,
+                        int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
+    if (!sizes_ok(T, K, E) || !ncap_ok(N_cap, T, K)) return MOE_ERR_INVALID_ARG;
+    if (row_bytes <= 0 || row_bytes % 16 || row_bytes / 16 > INT32_MAX / 2) return MOE_ERR_INVALID_ARG;
+    if (aux_row_bytes < 0 || aux_row_bytes % 4 || aux_row_bytes > 65536) return MOE_ERR_INVALID_ARG;
+    if (aux_row_bytes > 0 && ((T > 0 && !aux) || (N_cap > 0 && !aux_perm))) return MOE_ERR_INVALID_ARG;
+    if (!expert_offsets || !workspace || !status) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !topk_idx || !flat_to_row)) return MOE_ERR_INVALID_ARG;
+    if (N_cap > 0 && (!x_perm || !row_to_flat)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(aux, 4) || !aligned(aux_perm, 4) ||
+        !aligned(topk_idx, 8) || !aligned(workspace, 16) || !aligned(expert_offsets, 4) ||
+        !aligned(row_to_flat, 4) || !aligned(flat_to_row, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    return finish(moe::launch_permute_payload(x, row_bytes, aux, aux_row_bytes, topk_idx, T, K, E,
+                                              expert_offsets, workspace, zero_pad, N_cap, x_perm,
+                                              aux_perm, row_to_flat, flat_to_row, status, stream));
+}
+
+int moe_combine_weighted_f32(const float* rows, int64_t N_cap, const int32_t* row_to_flat,
+                             const int32_t* flat_to_row, const void* weights, int weight_dtype,
+                             int T, int K, int H, int validate, float* out, int32_t* status,
+                             cudaStream_t stream) {
+    if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || H <= 0 || H % 4 ||
+        N_cap < 0 || N_cap > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (weight_dtype != MOE_DTYPE_F32 && weight_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (!status) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!flat_to_row || !out)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && N_cap > 0 && !rows) return MOE_ERR_INVALID_ARG;
+    if (validate && N_cap > 0 && !row_to_flat) return MOE_ERR_INVALID_ARG;
+    const size_t wal = weight_dtype == MOE_DTYPE_F32 ? 4 : 2;
+    if (!aligned(rows, 16) || !aligned(out, 16) || !aligned(flat_to_row, 4) ||
+        !aligned(row_to_flat, 4) || !aligned(weights, wal) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0 && !validate) return MOE_OK;
+    return finish(moe::launch_combine_f32(rows, N_cap, row_to_flat, flat_to_row, weights,
+                                          weight_dtype, T, K, H, validate, out, status, stream));
+}
+
+int moe_combine_backward_f32(const float* grad_out, const float* rows, int64_t N_cap,
+                             const int32_t* row_to_flat, const int32_t* flat_to_row,
+                             const void* weights, int weight_dtype, int T, int K, int H,
+                             const int32_t* expert_offsets, int E, int zero_pad,
+                             float* grad_rows, void* grad_weights, int32_t* status,
+                             cudaStream_t stream) {
+    if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || H <= 0 || H % 4 ||
+        N_cap < 0 || N_cap > INT32_MAX || E < 1 || E > MOE_MAX_E)
+        return MOE_ERR_INVALID_ARG;
+    if (weight_dtype != MOE_DTYPE_F32 && weight_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (!status || !expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!grad_out || !flat_to_row || !weights)) return MOE_ERR_INVALID_ARG;
+    if (N_cap > 0 && (!rows || !grad_rows)) return MOE_ERR_INVALID_ARG;
+    if (zero_pad && N_cap > 0 && !row_to_flat) return MOE_ERR_INVALID_ARG;
+    const size_t wal = weight_dtype == MOE_DTYPE_F32 ? 4 : 2;
+    if (!aligned(grad_out, 16) || !aligned(rows, 16) || !aligned(grad_rows, 16) ||
+        !aligned(flat_to_row, 4) || !aligned(row_to_flat, 4) || !aligned(weights, wal) ||
+        !aligned(grad_weights, wal) || !aligned(expert_offsets, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0 && !zero_pad) return MOE_OK;
+    return finish(moe::launch_combine_backward_f32(grad_out, rows, N_cap, row_to_flat, flat_to_row,
+                                                   weights, weight_dtype, T, K, H, expert_offsets,
+                                                   E, zero_pad, grad_rows, grad_weights, status,
+                                                   stream));
+}
+
 int moe_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
                            int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
     if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || N < 0 || N > INT32_MAX)

@@ -27,16 +27,40 @@
 
 namespace moe {
 
+// Row element types.  A 16-byte vector holds kPer elements; unpack widens
+// them to fp32 exactly, pack rounds fp32 values to the row type (RNE for
+// bf16, nothing for fp32), prod is the exact product of a gradient and a row
+// element in fp64 (bf16 x bf16 is exact already in fp32; fp32 x fp32 is exact
+// in fp64).  The fp32 rows are the activation-dtype-fp32 case of the
+// DeepSpeed folding PR's Tests ("fp32 and bf16 rows").
+struct RowBf16 {
+    static constexpr int kPer = 8;
+    __device__ __forceinline__ static void unpack(const uint4& v, float (&f)[8]) { unpack8(v, f); }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[8]) { return pack8(f); }
+    __device__ __forceinline__ static double prod(float g, float y) { return (double)__fmul_rn(g, y); }
+};
+struct RowF32 {
+    static constexpr int kPer = 4;
+    __device__ __forceinline__ static void unpack(const uint4& v, float (&f)[4]) {
+        f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[4]) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                          __float_as_uint(f[3]));
+    }
+    __device__ __forceinline__ static double prod(float g, float y) { return (double)g * (double)y; }
+};
+
 // ------------------------------------------------- forward, any K ---
 // One warp per token; for each column chunk of 32 x U vectors the slots are
 // visited in order (any K up to MOE_MAX_K).
-template <int U, bool VALIDATE>
+template <typename Tr, int U, bool VALIDATE>
 __global__ void __launch_bounds__(kBlock)
-combine_kernel(const uint16_t* __restrict__ rows, int64_t N_cap, const int32_t* __restrict__ r2f,
+combine_kernel(const uint4* __restrict__ rows, int64_t N_cap, const int32_t* __restrict__ r2f,
                const int32_t* __restrict__ f2r, const void* __restrict__ w, int wdtype, int T,
-               int K, int H, uint16_t* __restrict__ out, int32_t* __restrict__ status) {
+               int K, int n16, uint4* __restrict__ out, int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n16 = H >> 3;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     int bad = 0;
 
@@ -55,35 +79,35 @@ combine_kernel(const uint16_t* __restrict__ rows, int64_t N_cap, const int32_t* 
             }
             myrow = r;
         }
-        uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * H);
+        uint4* dst = out + (size_t)t * n16;
         // Warp-uniform trip count: the shuffles inside need all 32 lanes.
         for (int c0 = 0; c0 < n16; c0 += 32 * U) {
             const int c = c0 + lane;
-            float acc[U][8];
+            float acc[U][Tr::kPer];
 #pragma unroll
             for (int u = 0; u < U; ++u)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+                for (int i = 0; i < Tr::kPer; ++i) acc[u][i] = 0.f;
             for (int k = 0; k < K; ++k) {
                 const int r = __shfl_sync(kFull, myrow, k);
                 const float wv = __shfl_sync(kFull, myw, k);
                 if (r < 0) continue;
-                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)r * H);
+                const uint4* src = rows + (size_t)r * n16;
                 uint4 v[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u)
                     v[u] = (c + 32 * u < n16) ? ld_stream(src + c + 32 * u) : zero;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    float y[8];
-                    unpack8(v[u], y);
+                    float y[Tr::kPer];
+                    Tr::unpack(v[u], y);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[u][i] = __fmaf_rn(wv, y[i], acc[u][i]);
+                    for (int i = 0; i < Tr::kPer; ++i) acc[u][i] = __fmaf_rn(wv, y[i], acc[u][i]);
                 }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                if (c + 32 * u < n16) st_vec(dst + c + 32 * u, pack8(acc[u]));
+                if (c + 32 * u < n16) st_vec(dst + c + 32 * u, Tr::pack(acc[u]));
         }
     }
 
@@ -116,14 +140,13 @@ combine_kernel(const uint16_t* __restrict__ rows, int64_t N_cap, const int32_t* 
 #define MOE_COMBINE_D 4
 #endif
 
-template <int KT, int U, int D, bool VALIDATE>
+template <typename Tr, int KT, int U, int D, bool VALIDATE>
 __global__ void __launch_bounds__(kBlock)
-combine_slots_kernel(const uint16_t* __restrict__ rows, int64_t N_cap,
+combine_slots_kernel(const uint4* __restrict__ rows, int64_t N_cap,
                      const int32_t* __restrict__ r2f, const int32_t* __restrict__ f2r,
-                     const void* __restrict__ w, int wdtype, int T, int H,
-                     uint16_t* __restrict__ out, int32_t* __restrict__ status) {
+                     const void* __restrict__ w, int wdtype, int T, int n16,
+                     uint4* __restrict__ out, int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n16 = H >> 3;
     const int chunks = (n16 + 32 * U - 1) / (32 * U);
     const int64_t n_items = (int64_t)T * chunks;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
@@ -158,40 +181,40 @@ combine_slots_kernel(const uint16_t* __restrict__ rows, int64_t N_cap,
         uint4 ring[D][U];
 #pragma unroll
         for (int k = 0; k < D && k < KT; ++k) {
-            const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[k] < 0 ? 0 : rk[k]) * H);
+            const uint4* src = rows + (size_t)(rk[k] < 0 ? 0 : rk[k]) * n16;
 #pragma unroll
             for (int u = 0; u < U; ++u)
                 ring[k][u] = (rk[k] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
         }
-        float acc[U][8];
+        float acc[U][Tr::kPer];
 #pragma unroll
         for (int u = 0; u < U; ++u)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+            for (int i = 0; i < Tr::kPer; ++i) acc[u][i] = 0.f;
 #pragma unroll
         for (int k = 0; k < KT; ++k) {
             const int slot = k % D;
             if (rk[k] >= 0) {
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    float y[8];
-                    unpack8(ring[slot][u], y);
+                    float y[Tr::kPer];
+                    Tr::unpack(ring[slot][u], y);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[u][i] = __fmaf_rn(wk[k], y[i], acc[u][i]);
+                    for (int i = 0; i < Tr::kPer; ++i) acc[u][i] = __fmaf_rn(wk[k], y[i], acc[u][i]);
                 }
             }
             if (k + D < KT) {
                 const int kn = k + D;
-                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[kn] < 0 ? 0 : rk[kn]) * H);
+                const uint4* src = rows + (size_t)(rk[kn] < 0 ? 0 : rk[kn]) * n16;
 #pragma unroll
                 for (int u = 0; u < U; ++u)
                     ring[slot][u] = (rk[kn] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
             }
         }
-        uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * H);
+        uint4* dst = out + (size_t)t * n16;
 #pragma unroll
         for (int u = 0; u < U; ++u)
-            if (v0 + 32 * u < n16) st_vec(dst + v0 + 32 * u, pack8(acc[u]));
+            if (v0 + 32 * u < n16) st_vec(dst + v0 + 32 * u, Tr::pack(acc[u]));
     }
 
     if (VALIDATE) {
@@ -209,15 +232,15 @@ combine_slots_kernel(const uint16_t* __restrict__ rows, int64_t N_cap,
 // ------------------------------------------------ backward, any K ---
 // One warp per token, one slot at a time over the whole row (g is re-read
 // per slot from cache); the weight gradient is reduced per slot.
+template <typename Tr>
 __global__ void __launch_bounds__(kBlock)
-combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ rows,
+combine_bwd_kernel(const uint4* __restrict__ g, const uint4* __restrict__ rows,
                    int64_t N_cap, const int32_t* __restrict__ r2f,
                    const int32_t* __restrict__ f2r, const void* __restrict__ w, int wdtype, int T,
-                   int K, int H, const int32_t* __restrict__ offsets, int E, int zero_pad,
-                   uint16_t* __restrict__ grad_rows, void* __restrict__ grad_w,
+                   int K, int n16, const int32_t* __restrict__ offsets, int E, int zero_pad,
+                   uint4* __restrict__ grad_rows, void* __restrict__ grad_w,
                    int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n16 = H >> 3;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     int bad = 0;
 
@@ -235,26 +258,26 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
             }
             myrow = r;
         }
-        const uint4* gsrc = reinterpret_cast<const uint4*>(g + (size_t)t * H);
+        const uint4* gsrc = g + (size_t)t * n16;
         for (int k = 0; k < K; ++k) {
             const int r = __shfl_sync(kFull, myrow, k);
             const float wv = __shfl_sync(kFull, myw, k);
             double dk = 0.0;
             if (r >= 0) {
-                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)r * H);
-                uint4* dst = reinterpret_cast<uint4*>(grad_rows + (size_t)r * H);
+                const uint4* src = rows + (size_t)r * n16;
+                uint4* dst = grad_rows + (size_t)r * n16;
                 for (int c = lane; c < n16; c += 32) {
-                    float gf[8], yf[8], o[8];
-                    unpack8(gsrc[c], gf);
-                    unpack8(ld_stream(src + c), yf);
+                    float gf[Tr::kPer], yf[Tr::kPer], o[Tr::kPer];
+                    Tr::unpack(gsrc[c], gf);
+                    Tr::unpack(ld_stream(src + c), yf);
                     double part = 0.0;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        part += (double)__fmul_rn(gf[i], yf[i]);   // exact: bf16 x bf16
+                    for (int i = 0; i < Tr::kPer; ++i) {
+                        part += Tr::prod(gf[i], yf[i]);   // exact
                         o[i] = __fmul_rn(wv, gf[i]);
                     }
                     dk += part;
-                    st_vec(dst + c, pack8(o));
+                    st_vec(dst + c, Tr::pack(o));
                 }
             }
 #pragma unroll
@@ -284,7 +307,7 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
             while (m) {
                 const int b = __ffs(m) - 1;
                 m &= m - 1;
-                uint4* dst = reinterpret_cast<uint4*>(grad_rows + (size_t)(base + b) * H);
+                uint4* dst = grad_rows + (size_t)(base + b) * n16;
                 for (int c = lane; c < n16; c += 32) st_vec(dst + c, zero);
             }
         }
@@ -303,16 +326,15 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
 #define MOE_BWD_MIN_BLOCKS 2
 #endif
 
-template <int KT, int U, int D>
+template <typename Tr, int KT, int U, int D>
 __global__ void __launch_bounds__(kBlock, MOE_BWD_MIN_BLOCKS)
-combine_bwd_slots_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ rows,
+combine_bwd_slots_kernel(const uint4* __restrict__ g, const uint4* __restrict__ rows,
                          int64_t N_cap, const int32_t* __restrict__ r2f,
                          const int32_t* __restrict__ f2r, const void* __restrict__ w, int wdtype,
-                         int T, int H, const int32_t* __restrict__ offsets, int E, int zero_pad,
-                         uint16_t* __restrict__ grad_rows, void* __restrict__ grad_w,
+                         int T, int n16, const int32_t* __restrict__ offsets, int E, int zero_pad,
+                         uint4* __restrict__ grad_rows, void* __restrict__ grad_w,
                          int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n16 = H >> 3;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     int bad = 0;
 
@@ -339,7 +361,7 @@ combine_bwd_slots_kernel(const uint16_t* __restrict__ g, const uint16_t* __restr
             wk[k] = __shfl_sync(kFull, myw, k);
             dot[k] = 0.0;
         }
-        const uint4* gsrc = reinterpret_cast<const uint4*>(g + (size_t)t * H);
+        const uint4* gsrc = g + (size_t)t * n16;
         for (int c0 = 0; c0 < n16; c0 += 32 * U) {
             const int v0 = c0 + lane;
             uint4 gv[U];
@@ -348,7 +370,7 @@ combine_bwd_slots_kernel(const uint16_t* __restrict__ g, const uint16_t* __restr
             uint4 ring[D][U];
 #pragma unroll
             for (int k = 0; k < D && k < KT; ++k) {
-                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[k] < 0 ? 0 : rk[k]) * H);
+                const uint4* src = rows + (size_t)(rk[k] < 0 ? 0 : rk[k]) * n16;
 #pragma unroll
                 for (int u = 0; u < U; ++u)
                     ring[k][u] = (rk[k] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
@@ -357,26 +379,26 @@ combine_bwd_slots_kernel(const uint16_t* __restrict__ g, const uint16_t* __restr
             for (int k = 0; k < KT; ++k) {
                 const int slot = k % D;
                 if (rk[k] >= 0) {
-                    uint4* dst = reinterpret_cast<uint4*>(grad_rows + (size_t)rk[k] * H);
+                    uint4* dst = grad_rows + (size_t)rk[k] * n16;
                     double part = 0.0;
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
                         if (v0 + 32 * u >= n16) continue;
-                        float gf[8], yf[8], o[8];
-                        unpack8(gv[u], gf);
-                        unpack8(ring[slot][u], yf);
+                        float gf[Tr::kPer], yf[Tr::kPer], o[Tr::kPer];
+                        Tr::unpack(gv[u], gf);
+                        Tr::unpack(ring[slot][u], yf);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            part += (double)__fmul_rn(gf[i], yf[i]);   // exact: bf16 x bf16
+                        for (int i = 0; i < Tr::kPer; ++i) {
+                            part += Tr::prod(gf[i], yf[i]);   // exact
                             o[i] = __fmul_rn(wk[k], gf[i]);
                         }
-                        st_vec(dst + v0 + 32 * u, pack8(o));
+                        st_vec(dst + v0 + 32 * u, Tr::pack(o));
                     }
                     dot[k] += part;
                 }
                 if (k + D < KT) {
                     const int kn = k + D;
-                    const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)(rk[kn] < 0 ? 0 : rk[kn]) * H);
+                    const uint4* src = rows + (size_t)(rk[kn] < 0 ? 0 : rk[kn]) * n16;
 #pragma unroll
                     for (int u = 0; u < U; ++u)
                         ring[slot][u] = (rk[kn] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
@@ -413,7 +435,7 @@ combine_bwd_slots_kernel(const uint16_t* __restrict__ g, const uint16_t* __restr
             while (m) {
                 const int b = __ffs(m) - 1;
                 m &= m - 1;
-                uint4* dst = reinterpret_cast<uint4*>(grad_rows + (size_t)(base + b) * H);
+                uint4* dst = grad_rows + (size_t)(base + b) * n16;
                 for (int c = lane; c < n16; c += 32) st_vec(dst + c, zero);
             }
         }
@@ -423,11 +445,12 @@ combine_bwd_slots_kernel(const uint16_t* __restrict__ g, const uint16_t* __restr
 
 // ------------------------------------------------------------ launchers ---
 
-template <bool V>
-static void launch_combine_t(int K, int grid, cudaStream_t st, const uint16_t* rows, int64_t N_cap,
+template <typename Tr, bool V>
+static void launch_combine_t(int K, int grid, cudaStream_t st, const uint4* rows, int64_t N_cap,
                              const int32_t* r2f, const int32_t* f2r, const void* w, int wd, int T,
-                             int H, uint16_t* out, int32_t* status) {
-    combine_kernel<2, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, K, H, out, status);
+                             int n16, uint4* out, int32_t* status) {
+    combine_kernel<Tr, 2, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, K, n16, out,
+                                                      status);
 }
 
 // Enough warps for one token each (up to 8 resident CTAs per SM), and, when a
@@ -446,30 +469,32 @@ static int grid_tokens_and_rows(int T, int64_t N_cap, bool sweep_rows, int per_s
     return want < 1 ? 1 : (int)want;
 }
 
-template <bool V>
-static void launch_slots_t(int K, int grid, cudaStream_t st, const uint16_t* rows, int64_t N_cap,
+#define MOE_SLOTS_ARGS rows, N_cap, r2f, f2r, w, wd, T, n16, out, status
+
+template <typename Tr, bool V>
+static void launch_slots_t(int K, int grid, cudaStream_t st, const uint4* rows, int64_t N_cap,
                            const int32_t* r2f, const int32_t* f2r, const void* w, int wd, int T,
-                           int H, uint16_t* out, int32_t* status) {
+                           int n16, uint4* out, int32_t* status) {
     constexpr int U = MOE_COMBINE_U, D = MOE_COMBINE_D;
     // Small K: wider chunks keep as many vectors in flight per lane.
     switch (K) {
-        case 1: combine_slots_kernel<1, 4 * U, 1, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
-        case 2: combine_slots_kernel<2, 2 * U, 2, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
-        case 3: combine_slots_kernel<3, U, (D < 3 ? D : 3), V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
-        case 4: combine_slots_kernel<4, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
-        case 5: combine_slots_kernel<5, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
-        case 6: combine_slots_kernel<6, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
-        case 7: combine_slots_kernel<7, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
-        default: combine_slots_kernel<8, U, D, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, H, out, status); break;
+        case 1: combine_slots_kernel<Tr, 1, 4 * U, 1, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
+        case 2: combine_slots_kernel<Tr, 2, 2 * U, 2, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
+        case 3: combine_slots_kernel<Tr, 3, U, (D < 3 ? D : 3), V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
+        case 4: combine_slots_kernel<Tr, 4, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
+        case 5: combine_slots_kernel<Tr, 5, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
+        case 6: combine_slots_kernel<Tr, 6, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
+        case 7: combine_slots_kernel<Tr, 7, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
+        default: combine_slots_kernel<Tr, 8, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
     }
 }
 
-cudaError_t launch_combine(const uint16_t* rows, int64_t N_cap, const int32_t* row_to_flat,
-                           const int32_t* flat_to_row, const void* weights, int weight_dtype,
-                           int T, int K, int H, int validate, uint16_t* out, int32_t* status,
-                           cudaStream_t stream) {
+template <typename Tr>
+static cudaError_t launch_combine_rows(const uint4* rows, int64_t N_cap, const int32_t* r2f,
+                                       const int32_t* f2r, const void* w, int wd, int T, int K,
+                                       int n16, int validate, uint4* out, int32_t* status,
+                                       cudaStream_t stream) {
     if (K <= 8) {
-        const int n16 = H >> 3;
         const int u = K == 1 ? 4 * MOE_COMBINE_U : (K == 2 ? 2 * MOE_COMBINE_U : MOE_COMBINE_U);
         const int chunks = (n16 + 32 * u - 1) / (32 * u);
         const int64_t items = (int64_t)T * chunks;
@@ -484,37 +509,50 @@ cudaError_t launch_combine(const uint16_t* rows, int64_t N_cap, const int32_t* r
         }
         const int grid = (int)(want > cap ? cap : (want < 1 ? 1 : want));
         if (validate)
-            launch_slots_t<true>(K, grid, stream, rows, N_cap, row_to_flat, flat_to_row, weights,
-                                 weight_dtype, T, H, out, status);
+            launch_slots_t<Tr, true>(K, grid, stream, rows, N_cap, r2f, f2r, w, wd, T, n16, out,
+                                     status);
         else
-            launch_slots_t<false>(K, grid, stream, rows, N_cap, row_to_flat, flat_to_row, weights,
-                                  weight_dtype, T, H, out, status);
+            launch_slots_t<Tr, false>(K, grid, stream, rows, N_cap, r2f, f2r, w, wd, T, n16, out,
+                                      status);
         return cudaGetLastError();
     }
     const int grid = grid_tokens_and_rows(T, N_cap, validate != 0);
     if (validate)
-        launch_combine_t<true>(K, grid, stream, rows, N_cap, row_to_flat, flat_to_row, weights,
-                               weight_dtype, T, H, out, status);
+        launch_combine_t<Tr, true>(K, grid, stream, rows, N_cap, r2f, f2r, w, wd, T, n16, out,
+                                   status);
     else
-        launch_combine_t<false>(K, grid, stream, rows, N_cap, row_to_flat, flat_to_row, weights,
-                                weight_dtype, T, H, out, status);
+        launch_combine_t<Tr, false>(K, grid, stream, rows, N_cap, r2f, f2r, w, wd, T, n16, out,
+                                    status);
     return cudaGetLastError();
 }
 
+cudaError_t launch_combine(const uint16_t* rows, int64_t N_cap, const int32_t* row_to_flat,
+                           const int32_t* flat_to_row, const void* weights, int weight_dtype,
+                           int T, int K, int H, int validate, uint16_t* out, int32_t* status,
+                           cudaStream_t stream) {
+    return launch_combine_rows<RowBf16>(reinterpret_cast<const uint4*>(rows), N_cap, row_to_flat,
+                                        flat_to_row, weights, weight_dtype, T, K, H / 8, validate,
+                                        reinterpret_cast<uint4*>(out), status, stream);
+}
+
+cudaError_t launch_combine_f32(const float* rows, int64_t N_cap, const int32_t* row_to_flat,
+                               const int32_t* flat_to_row, const void* weights, int weight_dtype,
+                               int T, int K, int H, int validate, float* out, int32_t* status,
+                               cudaStream_t stream) {
+    return launch_combine_rows<RowF32>(reinterpret_cast<const uint4*>(rows), N_cap, row_to_flat,
+                                       flat_to_row, weights, weight_dtype, T, K, H / 4, validate,
+                                       reinterpret_cast<uint4*>(out), status, stream);
+}
+
 #define MOE_BWD_SLOT_ARGS                                                                      \
-    grad_out, rows, N_cap, row_to_flat, flat_to_row, weights, weight_dtype, T, H, expert_offsets,  \
-        E, zero_pad, grad_rows, grad_weights, status
+    g, rows, N_cap, r2f, f2r, w, wd, T, n16, offsets, E, zero_pad, grad_rows, grad_w, status
 
-#define MOE_BWD_ARGS                                                                           \
-    grad_out, rows, N_cap, row_to_flat, flat_to_row, weights, weight_dtype, T, K, H,           \
-        expert_offsets, E, zero_pad, grad_rows, grad_weights, status
-
-cudaError_t launch_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t N_cap,
-                                    const int32_t* row_to_flat, const int32_t* flat_to_row,
-                                    const void* weights, int weight_dtype, int T, int K, int H,
-                                    const int32_t* expert_offsets, int E, int zero_pad,
-                                    uint16_t* grad_rows, void* grad_weights, int32_t* status,
-                                    cudaStream_t stream) {
+template <typename Tr>
+static cudaError_t launch_backward_rows(const uint4* g, const uint4* rows, int64_t N_cap,
+                                        const int32_t* r2f, const int32_t* f2r, const void* w,
+                                        int wd, int T, int K, int n16, const int32_t* offsets,
+                                        int E, int zero_pad, uint4* grad_rows, void* grad_w,
+                                        int32_t* status, cudaStream_t stream) {
     const int grid = grid_tokens_and_rows(T, N_cap, zero_pad != 0, MOE_BWD_GRID_PER_SM);
 #ifndef MOE_BWD_U
 #define MOE_BWD_U MOE_COMBINE_U
@@ -524,17 +562,45 @@ cudaError_t launch_combine_backward(const uint16_t* grad_out, const uint16_t* ro
 #endif
     constexpr int U = MOE_BWD_U, D = MOE_BWD_D;
     switch (K) {
-        case 1: combine_bwd_slots_kernel<1, 4 * U, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 2: combine_bwd_slots_kernel<2, 2 * U, 2><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 3: combine_bwd_slots_kernel<3, U, (D < 3 ? D : 3)><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 4: combine_bwd_slots_kernel<4, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 5: combine_bwd_slots_kernel<5, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 6: combine_bwd_slots_kernel<6, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 7: combine_bwd_slots_kernel<7, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 8: combine_bwd_slots_kernel<8, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        default: combine_bwd_kernel<<<grid, kBlock, 0, stream>>>(MOE_BWD_ARGS); break;
+        case 1: combine_bwd_slots_kernel<Tr, 1, 4 * U, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 2: combine_bwd_slots_kernel<Tr, 2, 2 * U, 2><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 3: combine_bwd_slots_kernel<Tr, 3, U, (D < 3 ? D : 3)><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 4: combine_bwd_slots_kernel<Tr, 4, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 5: combine_bwd_slots_kernel<Tr, 5, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 6: combine_bwd_slots_kernel<Tr, 6, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 7: combine_bwd_slots_kernel<Tr, 7, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 8: combine_bwd_slots_kernel<Tr, 8, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        default:
+            combine_bwd_kernel<Tr><<<grid, kBlock, 0, stream>>>(g, rows, N_cap, r2f, f2r, w, wd, T,
+                                                                K, n16, offsets, E, zero_pad,
+                                                                grad_rows, grad_w, status);
+            break;
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t N_cap,
+                                    const int32_t* row_to_flat, const int32_t* flat_to_row,
+                                    const void* weights, int weight_dtype, int T, int K, int H,
+                                    const int32_t* expert_offsets, int E, int zero_pad,
+                                    uint16_t* grad_rows, void* grad_weights, int32_t* status,
+                                    cudaStream_t stream) {
+    return launch_backward_rows<RowBf16>(
+        reinterpret_cast<const uint4*>(grad_out), reinterpret_cast<const uint4*>(rows), N_cap,
+        row_to_flat, flat_to_row, weights, weight_dtype, T, K, H / 8, expert_offsets, E, zero_pad,
+        reinterpret_cast<uint4*>(grad_rows), grad_weights, status, stream);
+}
+
+cudaError_t launch_combine_backward_f32(const float* grad_out, const float* rows, int64_t N_cap,
+                                        const int32_t* row_to_flat, const int32_t* flat_to_row,
+                                        const void* weights, int weight_dtype, int T, int K, int H,
+                                        const int32_t* expert_offsets, int E, int zero_pad,
+                                        float* grad_rows, void* grad_weights, int32_t* status,
+                                        cudaStream_t stream) {
+    return launch_backward_rows<RowF32>(
+        reinterpret_cast<const uint4*>(grad_out), reinterpret_cast<const uint4*>(rows), N_cap,
+        row_to_flat, flat_to_row, weights, weight_dtype, T, K, H / 4, expert_offsets, E, zero_pad,
+        reinterpret_cast<uint4*>(grad_rows), grad_weights, status, stream);
 }
 
 }  // namespace moe

@@ -88,6 +88,13 @@ cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, in
                            int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat,
                            int32_t* flat_to_row, int32_t* status, cudaStream_t stream);
 
+cudaError_t launch_permute_payload(const void* x, int64_t row_bytes, const void* aux,
+                                   int64_t aux_row_bytes, const int64_t* topk_idx, int T, int K,
+                                   int E, const int32_t* expert_offsets, const void* workspace,
+                                   int zero_pad, int64_t N_cap, void* x_perm, void* aux_perm,
+                                   int32_t* row_to_flat, int32_t* flat_to_row, int32_t* status,
+                                   cudaStream_t stream);
+
 cudaError_t launch_expert_scale(const uint16_t* rows, int64_t N_cap, const int32_t* expert_offsets,
                                 const int32_t* tokens_per_expert, int E, int H,
                                 const float* scales, uint16_t* out, int32_t* status,
@@ -97,6 +104,18 @@ cudaError_t launch_combine(const uint16_t* rows, int64_t N_cap, const int32_t* r
                            const int32_t* flat_to_row, const void* weights, int weight_dtype,
                            int T, int K, int H, int validate, uint16_t* out, int32_t* status,
                            cudaStream_t stream);
+
+cudaError_t launch_combine_f32(const float* rows, int64_t N_cap, const int32_t* row_to_flat,
+                               const int32_t* flat_to_row, const void* weights, int weight_dtype,
+                               int T, int K, int H, int validate, float* out, int32_t* status,
+                               cudaStream_t stream);
+
+cudaError_t launch_combine_backward_f32(const float* grad_out, const float* rows, int64_t N_cap,
+                                        const int32_t* row_to_flat, const int32_t* flat_to_row,
+                                        const void* weights, int weight_dtype, int T, int K, int H,
+                                        const int32_t* expert_offsets, int E, int zero_pad,
+                                        float* grad_rows, void* grad_weights, int32_t* status,
+                                        cudaStream_t stream);
 
 cudaError_t launch_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
                                       int32_t* flat_to_row, int32_t* status, cudaStream_t stream);

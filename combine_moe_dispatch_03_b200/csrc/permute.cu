@@ -13,6 +13,11 @@
 // one read of every token row, K writes of it, the two row maps, and the
 // pad rows.  Work is cut into equal warp items (4 KB row pieces) and strided
 // over a grid of several CTAs per SM, so every warp moves the same bytes.
+//
+// Rows are opaque: a row is n16 16-byte vectors (bf16 rows: H/8; FP8 rows of
+// the (data, scales) tuple the DeepEP issue's dispatch accepts: H/16; fp32
+// rows: H/4).  With AUX, every token also owns a small aux row of 4-byte
+// words (the FP8 scales) that goes to the same K rows.
 #include "common.cuh"
 #include "internal.h"
 
@@ -23,12 +28,14 @@ namespace moe {
 // stored to the token's K rows -- then (pad row, piece) items.  The rows come
 // from the layout workspace: row(f) = off[e] + tile_base[e][tile(t)] +
 // in_rank[f]; the warp that handles piece 0 of a token also writes the
-// token's entries of both maps.  A final sweep marks the tail rows.
-template <int U>
+// token's entries of both maps (and, with AUX, copies the aux row).  A final
+// sweep marks the tail rows.
+template <int U, bool AUX>
 __global__ void __launch_bounds__(kBlock, 4)
-permute_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ topk, int T, int K,
-               int E, int H, const int32_t* __restrict__ offsets, const char* __restrict__ ws,
-               int zero_pad, int64_t N_cap, uint16_t* __restrict__ xp,
+permute_kernel(const uint4* __restrict__ x, int n16, const uint32_t* __restrict__ aux,
+               int aux_words, const int64_t* __restrict__ topk, int T, int K, int E,
+               const int32_t* __restrict__ offsets, const char* __restrict__ ws, int zero_pad,
+               int64_t N_cap, uint4* __restrict__ xp, uint32_t* __restrict__ auxp,
                int32_t* __restrict__ r2f, int32_t* __restrict__ f2r,
                int32_t* __restrict__ status) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -57,7 +64,6 @@ permute_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ topk,
     const int64_t N_pad = off[E];
     if (blockIdx.x == 0 && tid == 0 && N_pad > N_cap) atomicOr(status, MOE_ST_CAPACITY);
 
-    const int n16 = H >> 3;
     const int pieces = (n16 + 32 * U - 1) / (32 * U);
     const int64_t tok_items = (int64_t)T * pieces;
     const int64_t n_items = tok_items + (int64_t)P * pieces;
@@ -70,7 +76,7 @@ permute_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ topk,
             const int64_t t = item / pieces;
             const int p = (int)(item - t * pieces);
             const int v0 = p * 32 * U + lane;
-            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+            const uint4* src = x + (size_t)t * n16;
             uint4 v[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) v[u] = (v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
@@ -95,10 +101,15 @@ permute_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ topk,
             for (int k = 0; k < K; ++k) {
                 const int r = __shfl_sync(kFull, myrow, k);
                 if (r < 0) continue;
-                uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * H);
+                uint4* dst = xp + (size_t)r * n16;
 #pragma unroll
                 for (int u = 0; u < U; ++u)
                     if (v0 + 32 * u < n16) st_vec(dst + v0 + 32 * u, v[u]);
+                if (AUX && p == 0) {
+                    const uint32_t* asrc = aux + (size_t)t * aux_words;
+                    uint32_t* adst = auxp + (size_t)r * aux_words;
+                    for (int q = lane; q < aux_words; q += 32) adst[q] = __ldg(asrc + q);
+                }
             }
         } else {
             const int64_t pi = item - tok_items;
@@ -110,7 +121,9 @@ permute_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ topk,
             if (row < 0 || row >= N_cap) continue;
             if (p == 0 && lane == 0) r2f[row] = -1;
             if (!zero_pad) continue;
-            uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * H);
+            if (AUX && p == 0)
+                for (int wd = lane; wd < aux_words; wd += 32) auxp[(size_t)row * aux_words + wd] = 0u;
+            uint4* dst = xp + (size_t)row * n16;
 #pragma unroll
             for (int u = 0; u < U; ++u)
                 if (v0 + 32 * u < n16) st_vec(dst + v0 + 32 * u, zero);
@@ -124,10 +137,13 @@ permute_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ topk,
         r2f[row] = -1;
 }
 
-cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
-                           const int32_t* expert_offsets, const void* workspace, int zero_pad,
-                           int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat,
-                           int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
+template <bool AUX>
+static cudaError_t launch_rows(const uint4* x, int n16, const uint32_t* aux, int aux_words,
+                               const int64_t* topk_idx, int T, int K, int E,
+                               const int32_t* expert_offsets, const void* workspace, int zero_pad,
+                               int64_t N_cap, uint4* x_perm, uint32_t* aux_perm,
+                               int32_t* row_to_flat, int32_t* flat_to_row, int32_t* status,
+                               cudaStream_t stream) {
     // Enough CTAs to fill every SM several times over; the kernel strides
     // over its uniform items (token pieces, then pad-row pieces <= N_cap - A).
 #ifndef MOE_PERMUTE_U
@@ -135,7 +151,6 @@ cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, in
 #endif
     constexpr int U = MOE_PERMUTE_U;
     const int sms = sm_count_current_device();
-    const int n16 = H >> 3;
     const int64_t pieces = (n16 + 32 * U - 1) / (32 * U);
     const int64_t items = ((int64_t)T + (N_cap - (int64_t)T * K)) * pieces;
     int64_t grid = (items + kWarps - 1) / kWarps;
@@ -144,10 +159,40 @@ cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, in
 #endif
     if (grid > (int64_t)sms * MOE_PERMUTE_GRID_PER_SM) grid = (int64_t)sms * MOE_PERMUTE_GRID_PER_SM;
     if (grid < 1) grid = 1;
-    permute_kernel<U><<<(int)grid, kBlock, sizeof(int) * 2 * ((size_t)E + 1), stream>>>(
-        x, topk_idx, T, K, E, H, expert_offsets, static_cast<const char*>(workspace), zero_pad,
-        N_cap, x_perm, row_to_flat, flat_to_row, status);
+    permute_kernel<U, AUX><<<(int)grid, kBlock, sizeof(int) * 2 * ((size_t)E + 1), stream>>>(
+        x, n16, aux, aux_words, topk_idx, T, K, E, expert_offsets,
+        static_cast<const char*>(workspace), zero_pad, N_cap, x_perm, aux_perm, row_to_flat,
+        flat_to_row, status);
     return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
+                           const int32_t* expert_offsets, const void* workspace, int zero_pad,
+                           int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat,
+                           int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
+    return launch_rows<false>(reinterpret_cast<const uint4*>(x), H >> 3, nullptr, 0, topk_idx, T,
+                              K, E, expert_offsets, workspace, zero_pad, N_cap,
+                              reinterpret_cast<uint4*>(x_perm), nullptr, row_to_flat, flat_to_row,
+                              status, stream);
+}
+
+cudaError_t launch_permute_payload(const void* x, int64_t row_bytes, const void* aux,
+                                   int64_t aux_row_bytes, const int64_t* topk_idx, int T, int K,
+                                   int E, const int32_t* expert_offsets, const void* workspace,
+                                   int zero_pad, int64_t N_cap, void* x_perm, void* aux_perm,
+                                   int32_t* row_to_flat, int32_t* flat_to_row, int32_t* status,
+                                   cudaStream_t stream) {
+    const int n16 = (int)(row_bytes / 16);
+    const uint4* xs = static_cast<const uint4*>(x);
+    uint4* xd = static_cast<uint4*>(x_perm);
+    if (aux_row_bytes > 0 && aux_perm != nullptr)
+        return launch_rows<true>(xs, n16, static_cast<const uint32_t*>(aux),
+                                 (int)(aux_row_bytes / 4), topk_idx, T, K, E, expert_offsets,
+                                 workspace, zero_pad, N_cap, xd, static_cast<uint32_t*>(aux_perm),
+                                 row_to_flat, flat_to_row, status, stream);
+    return launch_rows<false>(xs, n16, nullptr, 0, topk_idx, T, K, E, expert_offsets, workspace,
+                              zero_pad, N_cap, xd, nullptr, row_to_flat, flat_to_row, status,
+                              stream);
 }
 
 }  // namespace moe

@@ -239,6 +239,62 @@ int moe_combine_weighted(const uint16_t* rows, int64_t N_cap, const int32_t* row
                          int T, int K, int H, int validate, uint16_t* out, int32_t* status,
                          cudaStream_t stream);
 
+/* ------------------------------------------------ payload and fp32 rows ---
+ * [DeepEP-272]: dispatch takes x either as a bf16 tensor or as an FP8 tuple
+ * (data, scales); [DS-8847] Tests: the fused restore on "fp32 and bf16 rows". */
+
+/* Dispatch of an opaque row payload: exactly moe_permute (same rows, maps,
+ * pad rows, tail, status bits and layout workspace) for rows of any byte
+ * width, plus an optional per-token aux row that goes to the same rows.
+ *
+ *   x_perm[row(f)] = x[t]         aux_perm[row(f)] = aux[t]
+ *
+ * FP8 tuple: x = e4m3 data [T,H] (row_bytes = H), aux = fp32 scales
+ * [T, H/128] (aux_row_bytes = 4*H/128).  fp32 rows: row_bytes = 4*H, aux NULL.
+ * In:  x [T, row_bytes] (16-byte aligned, row_bytes a positive multiple of
+ *      16); aux [T, aux_row_bytes] (4-byte aligned; aux_row_bytes a multiple
+ *      of 4, at most 65536; 0 means no aux payload and both aux pointers are
+ *      ignored).
+ * Out: x_perm [N_cap, row_bytes]; aux_perm [N_cap, aux_row_bytes];
+ *      row_to_flat [N_cap]; flat_to_row [T,K].  With zero_pad, pad rows of
+ *      both payloads are zero.  aux may be NULL only when T == 0 and
+ *      aux_perm only when N_cap == 0.
+ * Errors: MOE_ERR_INVALID_ARG as for moe_permute, or a row width outside
+ *         the rules above. */
+int moe_permute_payload(const void* x, int64_t row_bytes, const void* aux, int64_t aux_row_bytes,
+                        const int64_t* topk_idx, int T, int K, int E,
+                        const int32_t* expert_offsets, const void* workspace, int zero_pad,
+                        int64_t N_cap, void* x_perm, void* aux_perm, int32_t* row_to_flat,
+                        int32_t* flat_to_row, int32_t* status, cudaStream_t stream);
+
+/* fused_weighted_restore on fp32 rows: moe_combine_weighted with rows and
+ * out in fp32 (the activation dtype), the same FP32 fmaf chain in slot order
+ * and no final rounding:
+ *
+ *   out[t] = fmaf chain over k of (w[t,k], rows[flat_to_row[t*K+k]])
+ *
+ * Weights, validation and status exactly as moe_combine_weighted; H % 4 == 0
+ * (16-byte rows); rows and out 16-byte aligned. */
+int moe_combine_weighted_f32(const float* rows, int64_t N_cap, const int32_t* row_to_flat,
+                             const int32_t* flat_to_row, const void* weights, int weight_dtype,
+                             int T, int K, int H, int validate, float* out, int32_t* status,
+                             cudaStream_t stream);
+
+/* Backward of the fp32-row restore: moe_combine_backward with grad_out, rows
+ * and grad_rows in fp32:
+ *
+ *   grad_rows[flat_to_row[f]] = fp32(w[f] * g[t])      (one rounding)
+ *   grad_weights[f] = sum_h g[t,h] * rows[flat_to_row[f], h]
+ *
+ * fp32 x fp32 products are exact in fp64 and summed in fp64, then rounded
+ * once to the router dtype.  Everything else as moe_combine_backward. */
+int moe_combine_backward_f32(const float* grad_out, const float* rows, int64_t N_cap,
+                             const int32_t* row_to_flat, const int32_t* flat_to_row,
+                             const void* weights, int weight_dtype, int T, int K, int H,
+                             const int32_t* expert_offsets, int E, int zero_pad,
+                             float* grad_rows, void* grad_weights, int32_t* status,
+                             cudaStream_t stream);
+
 /* Scatter step of the folded restore ([DS-8847] Change: the rows of all
  * tensor-parallel peers are gathered together with ONE flat index per row,
  * token * top_k + slot; the routing data is scattered into [tokens, top_k];

@@ -2,7 +2,8 @@
 backward, on synthetic seeded inputs resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload qwen3|dsv3|dsv3_skew|mixtral|tiny]
+                    [--workload qwen3|dsv3|dsv3_skew|mixtral|tiny|page_k4|page_k8|
+                                page_k4_32k|page_k8_32k]
 
 Step (seven kernels, all through the C ABI of libmoe_dispatch.so):
   layout -> permute -> stand-in experts -> weighted combine

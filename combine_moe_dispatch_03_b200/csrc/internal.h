@@ -32,7 +32,7 @@ struct LayoutHeader {
 static_assert(sizeof(LayoutHeader) == 96, "header layout");
 
 constexpr int32_t kLayoutMagic = 0x4d6f4531;  // "MoE1"
-constexpr int kMaxTileAssign = 1024;          // TT * K <= this (32 warp chunks)
+constexpr int kMaxTileAssign = 2048;          // TT * K <= this (64 warp chunks)
 constexpr int kMaxTileChunks = kMaxTileAssign / 32;
 
 struct Geometry {

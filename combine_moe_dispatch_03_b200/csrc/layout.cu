@@ -219,30 +219,37 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
         warp_status_or(status, bad);
         __syncthreads();
 
-        // In-tile stable rank = same-expert assignments in earlier chunks +
-        // rank inside the chunk.
+        // Per expert, an exclusive scan of the chunk counts over the chunks
+        // (in place); its total is the tile's count of the expert.  The
+        // in-tile stable rank is then the scan at the assignment's chunk plus
+        // its rank inside the chunk.
+        for (int e = tid; e < E; e += kLThreads) {
+            int run = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int v = cnt[c * E + e];
+                cnt[c * E + e] = (uint16_t)run;
+                run += v;
+            }
+            tile_base[(size_t)e * n_tiles + j] = run;
+        }
+        __syncthreads();
         uint16_t* out_rank = in_rank + (size_t)t0 * K;
         for (int a = tid; a < na; a += kLThreads) {
             const int e = eidx[a];
-            if (e < 0) { out_rank[a] = 0xFFFFu; continue; }
-            int before = 0;
-            for (int c = 0; c < a / 32; ++c) before += cnt[c * E + e];
-            out_rank[a] = (uint16_t)(before + crank[a]);
-        }
-        for (int e = tid; e < E; e += kLThreads) {
-            int total = 0;
-            for (int c = 0; c < nchunks; ++c) total += cnt[c * E + e];
-            tile_base[(size_t)e * n_tiles + j] = total;
+            out_rank[a] = e < 0 ? (uint16_t)0xFFFFu : (uint16_t)(cnt[(a >> 5) * E + e] + crank[a]);
         }
         uint8_t* itr_tile = itr + (size_t)t0 * R;
         for (int idx = tid; idx < ntok * R; idx += kLThreads) {
             const int q = idx / R, r = idx - q * R;
             itr_tile[idx] = (uint8_t)((tokmask[q] >> r) & 1ull);
         }
-        for (int r = tid; r < R; r += kLThreads) {
+        // Distinct tokens of the tile per destination rank: a warp per rank.
+        for (int r = warp; r < R; r += kLWarps) {
             int n = 0;
-            for (int q = 0; q < ntok; ++q) n += (int)((tokmask[q] >> r) & 1ull);
-            tile_tpr[(size_t)r * n_tiles + j] = n;     // rank-major, like tile_base
+            for (int q = lane; q < ntok; q += 32) n += (int)((tokmask[q] >> r) & 1ull);
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) n += __shfl_xor_sync(kFull, n, d);
+            if (lane == 0) tile_tpr[(size_t)r * n_tiles + j] = n;   // rank-major, like tile_base
         }
     }
 

@@ -9,10 +9,11 @@ side can use it without touching the CUDA path.
 
 Workload shapes (tokens T, hidden H, experts E, logical ranks R, top_k K,
 alignment) follow the model families the AutoEP base PR presets (Mixtral,
-Qwen3-MoE, DeepSeek-V3; DeepSpeed AutoEP PR, "Supported presets") and the
+Qwen3-MoE, DeepSeek-V3; DeepSpeed AutoEP PR, "Supported presets"), the
 count-exchange measurement of the DeepSpeed PR "Derive AutoEP rank splits from
 the per-expert count exchange" (Measurements: 256 experts, 1024 tokens per
-rank, top_k 8, balanced / skewed token distributions).  No dataset is used.
+rank, top_k 8, balanced / skewed token distributions) and the benchmark table
+of the DeepSpeed fused-restore folding PR (page_*).  No dataset is used.
 
 Recipe (fixed draw order per config: x, logits, bias, zipf permutation,
 scales, grad_out):
@@ -73,6 +74,27 @@ CONFIGS = {
                     backward=True,
                     description="Qwen3-MoE-shaped fwd+bwd: T=16384 H=2048 E=128 (8x16) top-8 "
                                 "softmax, mild skew N(0,0.5) bias, align 16"),
+    # The benchmark shapes of the DeepSpeed PR "AutoEP: support
+    # combine_impl=fused_weighted_sum with AutoEP+AutoTP folding" (Benchmark:
+    # hidden 6144; top-4 of 128 and top-8 of 256 experts, the MiniMax-M3 and
+    # GLM-5.2 values; 8,192 and 32,768 tokens; random routing with distinct
+    # experts per token, FP32 weights).  No expert ranks, no group alignment.
+    "page_k4": Config("page_k4", T=8192, H=6144, E=128, R=1, K=4, align=1, seed=1005,
+                      router="sigmoid", backward=True,
+                      description="fused-restore benchmark shape (MiniMax-M3 values) fwd+bwd: "
+                                  "T=8192 H=6144 E=128 top-4 sigmoid-normalised"),
+    "page_k8": Config("page_k8", T=8192, H=6144, E=256, R=1, K=8, align=1, seed=1006,
+                      router="sigmoid", backward=True,
+                      description="fused-restore benchmark shape (GLM-5.2 values) fwd+bwd: "
+                                  "T=8192 H=6144 E=256 top-8 sigmoid-normalised"),
+    "page_k4_32k": Config("page_k4_32k", T=32768, H=6144, E=128, R=1, K=4, align=1, seed=1007,
+                          router="sigmoid", backward=True,
+                          description="fused-restore benchmark shape (MiniMax-M3 values) fwd+bwd: "
+                                      "T=32768 H=6144 E=128 top-4 sigmoid-normalised"),
+    "page_k8_32k": Config("page_k8_32k", T=32768, H=6144, E=256, R=1, K=8, align=1, seed=1008,
+                          router="sigmoid", backward=True,
+                          description="fused-restore benchmark shape (GLM-5.2 values) fwd+bwd: "
+                                      "T=32768 H=6144 E=256 top-8 sigmoid-normalised"),
 }
 
 

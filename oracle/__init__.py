@@ -76,6 +76,8 @@ def _load():
         lib.oracle_scatter_flat_index.restype = I
         lib.oracle_combine_backward.argtypes = [P, P, L, P, P, P, I, I, I, P, I, I, P, P]
         lib.oracle_combine_backward.restype = I
+        lib.oracle_restore_activation_dtype.argtypes = [P, L, P, P, P, I, I, I, P, P]
+        lib.oracle_restore_activation_dtype.restype = I
         lib.oracle_permute_payload.argtypes = [P, L, P, L, P, I, I, I, P, I, L, P, P, P, P]
         lib.oracle_permute_payload.restype = I
         lib.oracle_combine_f32.argtypes = [P, L, P, P, I, I, I, P, P]
@@ -321,4 +323,22 @@ def combine_backward_f32(grad_out: np.ndarray, rows: np.ndarray, row_to_flat: np
                                              _p(flat_to_row), _p(w), T, K, H, _p(expert_offsets), E,
                                              int(bool(zero_pad)), _p(grad_rows), _p(grad_w))
     return dict(grad_rows=grad_rows, grad_w=grad_w, status=st)
+
+
+def restore_activation_dtype(rows_bf16: np.ndarray, flat_to_row: np.ndarray, weights: np.ndarray,
+                             grad_out_bf16: np.ndarray | None = None) -> dict:
+    """The default (non-fused) folded restore: weights cast to bf16, every
+    product and top-k addition rounded to bf16; optional score gradient
+    through the bf16 weights.  An accuracy comparison only."""
+    rows_bf16 = _c(rows_bf16, np.uint16)
+    flat_to_row = _c(flat_to_row, np.int32)
+    T, K = flat_to_row.shape
+    N_cap, H = rows_bf16.shape
+    w = _c(np.asarray(weights, np.float32), np.float32)
+    g = None if grad_out_bf16 is None else _c(grad_out_bf16, np.uint16)
+    out = np.empty((T, H), np.uint16)
+    gw = np.empty((T, K), np.uint16) if g is not None else None
+    st = _load().oracle_restore_activation_dtype(_p(rows_bf16), N_cap, _p(flat_to_row), _p(w), _p(g),
+                                                 T, K, H, _p(out), _p(gw))
+    return dict(out=out, grad_w=gw, status=st)
 

@@ -550,3 +550,61 @@ int oracle_combine_backward_f32(const float* g, const float* rows, int64_t N_cap
     }
     return status;
 }
+
+/* The default folded restore of [DS-8847] (Problem: restore_combined casts
+ * the routing weights to the activation dtype and runs one index_add_ per
+ * top-k slot in bf16; Benchmark: its errors against FP64 and its score
+ * gradient "through bf16 weights"), kept only as an accuracy comparison for
+ * the fused restore.  Every product and every top-k addition is rounded to
+ * bf16; each operation is carried out in fp32 and rounded once (RNE), the way
+ * bf16 tensor arithmetic is:
+ *
+ *   wb = bf16(w);  acc = 0;
+ *   for k = 0..K-1:  acc = bf16(acc + bf16(wb[t,k] * y[row(t,k)]))
+ *
+ * and, when g != NULL, the score gradient through the bf16 weights:
+ *
+ *   grad_w[t,k] = bf16( sum_h bf16(g[t,h] * y[row(t,k),h]) )   (sum in fp64)
+ *
+ * Out-of-range slots contribute nothing (ORC_ROW_OOR); their gradient is 0. */
+int oracle_restore_activation_dtype(const uint16_t* rows, int64_t N_cap, const int32_t* flat_to_row,
+                                    const float* w, const uint16_t* g, int T, int K, int H,
+                                    uint16_t* out, uint16_t* grad_w) {
+    int status = 0;
+    for (int t = 0; t < T; ++t) {
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                int64_t f = (int64_t)t * K + k;
+                int64_t row = flat_to_row[f];
+                if (row < 0 || row >= N_cap) {
+                    status |= ORC_ROW_OOR;
+                    continue;
+                }
+                float wb = oracle_float_from_bf16(oracle_bf16_from_float(w[f]));
+                float y = oracle_float_from_bf16(rows[row * H + h]);
+                float p = oracle_float_from_bf16(oracle_bf16_from_float(wb * y));
+                acc = oracle_float_from_bf16(oracle_bf16_from_float(acc + p));
+            }
+            out[(int64_t)t * H + h] = oracle_bf16_from_float(acc);
+        }
+        if (!g || !grad_w) continue;
+        for (int k = 0; k < K; ++k) {
+            int64_t f = (int64_t)t * K + k;
+            int64_t row = flat_to_row[f];
+            if (row < 0 || row >= N_cap) {
+                grad_w[f] = 0;
+                continue;
+            }
+            double sum = 0.0;
+            for (int h = 0; h < H; ++h) {
+                float gv = oracle_float_from_bf16(g[(int64_t)t * H + h]);
+                float yv = oracle_float_from_bf16(rows[row * H + h]);
+                sum += (double)oracle_float_from_bf16(oracle_bf16_from_float(gv * yv));
+            }
+            grad_w[f] = oracle_bf16_from_float((float)sum);
+        }
+    }
+    return status;
+}
+

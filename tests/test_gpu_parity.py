@@ -38,7 +38,8 @@ def _check(inp, E, R, align, N_cap=None, **kw):
 
 # ------------------------------------------------------- seeded workloads ---
 
-@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "dsv3_skew", "qwen3"])
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "dsv3_skew", "qwen3", "page_k4",
+                                  "page_k8"])
 def test_config_full_size(name):
     """Every output of every call at the workload's full size, forward and
     backward, with the capacity and launch configuration the bench uses."""

@@ -95,7 +95,8 @@ def _layout_invariants(orc, topk, E, R, align):
     return lay
 
 
-@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "dsv3_skew", "qwen3"])
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "dsv3_skew", "qwen3", "page_k4",
+                                  "page_k8", "page_k4_32k", "page_k8_32k"])
 def test_layout_invariants_configs(orc, name):
     cfg = CONFIGS[name]
     inp = make_inputs(name, H=8)   # routing does not depend on H
@@ -705,3 +706,61 @@ def test_combine_backward_f32_finite_differences(orc):
     np.testing.assert_array_equal(bw["grad_rows"][real],
                                   (w.reshape(-1, 1).astype(np.float64) * gd[tok]).astype(np.float32))
     assert not bw["grad_rows"][: lay["expert_offsets"][-1]][r2f[: lay["expert_offsets"][-1]] < 0].any()
+
+
+# ------------------------------------- the default restore, for comparison ---
+
+def _default_table():
+    rows = []
+    with open(os.path.join(GOLDEN, "pages_default_restore_table.txt")) as fh:
+        for line in fh:
+            if line.startswith("#") or not line.strip():
+                continue
+            parts = [p.strip() for p in line.split("|")]
+            rows.append((tuple(int(v) for v in parts[0].split()), float(parts[1]), float(parts[2])))
+    return rows
+
+
+@pytest.mark.parametrize("which", [0, 2])
+def test_default_restore_error_matches_pages(orc, which):
+    """[DS-8847] Benchmark: rounding every product and top-k addition to bf16
+    (the default restore) gives the page's output error (3.58e-3 at top-4 of
+    128, 4.36e-3 at top-8 of 256) and, through bf16 weights, its score
+    gradient error (2.35e-3); the fused restore on the same inputs gives
+    1.66e-3.  Hidden size, top-k and experts as on the page; 256 tokens (the
+    errors are per element); independent bf16 rows per slot; weights are the
+    renormalised sigmoid scores of the selected experts (the gating of the
+    models the shapes come from)."""
+    (T0, K, E, H), out_err, score_err = _default_table()[which]
+    T = 256
+    wts = custom_inputs(T, 8, E, K, seed=70 + which, router="sigmoid")["weights"].numpy()
+    rng = np.random.default_rng(80 + which)
+    rows = orc.bf16_from_f32(rng.standard_normal((T * K, H)).astype(np.float32))
+    g = orc.bf16_from_f32(rng.standard_normal((T, H)).astype(np.float32))
+    f2r = np.arange(T * K, dtype=np.int32).reshape(T, K)
+    d = orc.restore_activation_dtype(rows, f2r, wts, g)
+    fused = orc.combine(rows, f2r, wts)
+    ref = fused["ref"]
+    e_def = rel_l2(orc.f32_from_bf16(d["out"]), ref)
+    e_fused = rel_l2(orc.f32_from_bf16(fused["seq"]), ref)
+    assert abs(e_def - out_err) / out_err < 0.05, e_def
+    assert abs(e_fused - 1.66e-3) / 1.66e-3 < 0.05, e_fused
+    gref = orc.combine_backward(g, rows, np.arange(T * K, dtype=np.int32), f2r, wts,
+                                np.array([0, T * K], np.int32))["grad_w"]
+    e_g = rel_l2(orc.f32_from_bf16(d["grad_w"]), gref)
+    assert abs(e_g - score_err) / score_err < 0.05, e_g
+
+
+def test_default_restore_hand_examples(orc):
+    """K = 1, w = 1: the row itself.  Three slots of weight 1 holding
+    1, 2^-8, 2^-8: each bf16 addition of 2^-8 to 1 is a tie that rounds back
+    to 1 (even), so the default restore returns 1.0, while the FP32 chain
+    keeps 1 + 2^-7 = 1.0078125, which bf16 represents exactly."""
+    rows = orc.bf16_from_f32(np.array([[1.5, -2.25, 3.0, 0.1]], np.float32))
+    d = orc.restore_activation_dtype(rows, np.zeros((1, 1), np.int32), np.ones((1, 1), np.float32))
+    np.testing.assert_array_equal(d["out"], rows)
+    rows = orc.bf16_from_f32(np.array([[1.0], [2.0 ** -8], [2.0 ** -8]], np.float32))
+    f2r = np.array([[0, 1, 2]], np.int32)
+    w = np.ones((1, 3), np.float32)
+    assert orc.f32_from_bf16(orc.restore_activation_dtype(rows, f2r, w)["out"])[0, 0] == 1.0
+    assert orc.f32_from_bf16(orc.combine(rows, f2r, w)["seq"])[0, 0] == 1.0078125

@@ -7,15 +7,20 @@
 
 namespace moe {
 
-// Layout workspace: [header | tile_base (E x n_tiles) | tile_tpr (R x n_tiles)
-// | expert_count (E) | in_rank (A = T*K, uint16)], each part 256-byte
-// aligned.  Tiles are runs of at most TT consecutive tokens that never
-// straddle two source ranks' token blocks, so per-rank sums are sums over
-// whole tiles.  tile_base[e][j] first holds the number of expert-e
-// assignments in tile j, then (after the scan) the number in all earlier
-// tiles: the stable base of tile j inside expert e's group.  in_rank[f] is
-// the number of earlier assignments of f's expert inside f's tile, so
+// Layout workspace: [header | expert_count (E) | splits_acc (R x R) |
+// tile_base (E x n_tiles) | tile_tpr (R x n_tiles) | in_rank (A = T*K,
+// uint16)], the parts after the accumulators 256-byte aligned.  Tiles are
+// runs of at most TT consecutive tokens that never straddle two source
+// ranks' token blocks, so per-rank sums are sums over whole tiles.
+// tile_base[e][j] first holds the number of expert-e assignments in tile j,
+// then (after the scan) the number in all earlier tiles: the stable base of
+// tile j inside expert e's group.  in_rank[f] is the number of earlier
+// assignments of f's expert inside f's tile, so
 //     row(f) = expert_offsets[e] + tile_base[e][tile(t)] + in_rank[f].
+// The bytes from the header's arrival counter to the end of splits_acc are
+// zeroed before every layout launch (one memset): the cooperative layout
+// accumulates per-expert totals and per-(source, destination) splits there
+// with atomics while it ranks its tiles.
 struct LayoutHeader {
     int64_t off_tile_base;     // byte offsets of the parts (so a reader needs no R)
     int64_t off_tile_tpr;
@@ -62,15 +67,19 @@ inline Geometry layout_geometry(int T, int K, int R) {
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t tile_base, tile_tpr, expert_count, in_rank, total;
+    size_t zero_begin, expert_count, splits_acc, zero_end;
+    size_t tile_base, tile_tpr, in_rank, total;
 };
 
 inline WsLayout workspace_layout(int E, int R, int n_tiles, int64_t A) {
     WsLayout w;
-    w.tile_base = align256(sizeof(LayoutHeader));
+    w.zero_begin = offsetof(LayoutHeader, done);
+    w.expert_count = align256(sizeof(LayoutHeader));
+    w.splits_acc = w.expert_count + sizeof(int32_t) * (size_t)E;
+    w.zero_end = w.splits_acc + sizeof(int32_t) * (size_t)R * (size_t)R;
+    w.tile_base = align256(w.zero_end);
     w.tile_tpr = w.tile_base + align256(sizeof(int32_t) * (size_t)E * (size_t)n_tiles);
-    w.expert_count = w.tile_tpr + align256(sizeof(int32_t) * (size_t)n_tiles * (size_t)R);
-    w.in_rank = w.expert_count + align256(sizeof(int32_t) * (size_t)E);
+    w.in_rank = w.tile_tpr + align256(sizeof(int32_t) * (size_t)n_tiles * (size_t)R);
     w.total = w.in_rank + align256(sizeof(uint16_t) * (size_t)A);
     return w;
 }

@@ -19,11 +19,15 @@
 //     source block (count matrix, tokens_per_rank).
 //   phase 3: padded exclusive offsets and splits.
 // When every tile's CTA fits on the GPU at once the launch is cooperative:
-// phases are separated by two grid barriers (bounded spins on a counter that
-// record MOE_ST_TIMEOUT instead of hanging) and phase 2 is spread over every
-// warp of the grid.  Otherwise the last CTA to arrive (an arrival counter, no
-// waiting) runs phases 2 and 3 alone.  The counter lives in the workspace
-// header and is zeroed by a 4-byte memset enqueued just before the kernel.
+// phase 1 also adds each tile's per-expert counts and per-destination-rank
+// sums into zeroed accumulators in the workspace (atomics), so one grid
+// barrier (a bounded spin on a counter that records MOE_ST_TIMEOUT instead
+// of hanging) separates phase 1 from everything else: after it, CTA 0 runs
+// phase 3 from the accumulated totals while the warps of the other CTAs scan
+// the rows, each lane holding its segment of a row in registers.  Otherwise
+// the last CTA to arrive (an arrival counter, no waiting) runs phases 2 and 3
+// alone.  The counter and the accumulators sit at the start of the workspace
+// and are zeroed by one memset enqueued just before the kernel.
 //
 // Bytes: reads topk_idx once (8*A), writes the [T,R] flags, in-tile ranks
 // (2*A) and O((E+R) * tiles) ints.
@@ -154,6 +158,64 @@ __device__ RowOut scan_row(int p, int E, int R, const Geometry& geo, int32_t* ti
     return o;
 }
 
+// Phase 2 for one row p in the cooperative path, where the grid has at
+// most kCoopMaxTiles tiles: each lane loads its segment of the row once into
+// registers (independent loads, one L2 round trip), then the same exclusive
+// scan and per-block sums as scan_row.
+constexpr int kCoopSeg = 5;
+constexpr int kCoopMaxTiles = 32 * kCoopSeg;
+
+__device__ void scan_row_regs(int p, int E, int R, const Geometry& geo, int32_t* tile_base,
+                              int32_t* tile_tpr, int* bs, int32_t* counts,
+                              int32_t* tokens_per_rank) {
+    const int lane = threadIdx.x & 31;
+    const int n_tiles = geo.n_tiles, El = E / R;
+    const bool is_expert = p < E;
+    int32_t* rowg = is_expert ? tile_base + (size_t)p * n_tiles
+                              : tile_tpr + (size_t)(p - E) * n_tiles;
+    for (int q = lane; q <= R; q += 32) bs[q] = 0;
+    __syncwarp();
+    const int seg = (n_tiles + 31) / 32;
+    const int j0 = min(lane * seg, n_tiles), j1 = min(j0 + seg, n_tiles);
+    int v[kCoopSeg];
+    int local = 0;
+#pragma unroll
+    for (int i = 0; i < kCoopSeg; ++i) {
+        v[i] = (j0 + i < j1) ? __ldcg(rowg + j0 + i) : 0;
+        local += v[i];
+    }
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int x = __shfl_up_sync(kFull, incl, d);
+        if (lane >= d) incl += x;
+    }
+    const int total = __shfl_sync(kFull, incl, 31);
+    int run = incl - local;
+#pragma unroll
+    for (int i = 0; i < kCoopSeg; ++i) {
+        const int jj = j0 + i;
+        if (jj < j1) {
+            if (is_expert) rowg[jj] = run;
+            if (jj % geo.tpb == 0) bs[jj / geo.tpb] = run;
+            run += v[i];
+        }
+    }
+    __syncwarp();
+    if (lane == 0) bs[R] = total;
+    __syncwarp();
+    if (is_expert) {
+        const int r = p / El, el = p - r * El;
+        for (int sb = lane; sb < R; sb += 32)
+            counts[((size_t)sb * R + r) * El + el] = bs[sb + 1] - bs[sb];
+    } else {
+        const int r = p - E;
+        for (int sb = lane; sb < R; sb += 32)
+            tokens_per_rank[(size_t)sb * R + r] = bs[sb + 1] - bs[sb];
+    }
+    __syncwarp();
+}
+
 __global__ void __launch_bounds__(kLThreads, 1)
 layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int align,
               Geometry geo, int32_t* __restrict__ tokens_per_expert, int32_t* __restrict__ counts,
@@ -163,6 +225,7 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int scratch[kLWarps + 1];
     __shared__ int am_last;
+    __shared__ int rank_sum[MOE_MAX_R];
     const int j = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int Tb = R > 0 ? T / R : 0, El = E / R;
@@ -170,6 +233,7 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
     int32_t* tile_base = reinterpret_cast<int32_t*>(ws + wl.tile_base);
     int32_t* tile_tpr = reinterpret_cast<int32_t*>(ws + wl.tile_tpr);
     int32_t* expert_count = reinterpret_cast<int32_t*>(ws + wl.expert_count);
+    int32_t* splits_acc = reinterpret_cast<int32_t*>(ws + wl.splits_acc);
     uint16_t* in_rank = reinterpret_cast<uint16_t*>(ws + wl.in_rank);
     LayoutHeader* hdr = reinterpret_cast<LayoutHeader*>(ws);
 
@@ -197,6 +261,7 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
 
         for (int q = tid; q < nchunks * E; q += kLThreads) cnt[q] = 0;
         for (int q = tid; q < ntok; q += kLThreads) tokmask[q] = 0ull;
+        if (tid < R) rank_sum[tid] = 0;
         __syncthreads();
 
         int bad = 0;
@@ -231,8 +296,13 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
                 run += v;
             }
             tile_base[(size_t)e * n_tiles + j] = run;
+            if (coop && run) {
+                atomicAdd(&expert_count[e], run);
+                atomicAdd(&rank_sum[e / El], run);
+            }
         }
         __syncthreads();
+        if (coop && tid < R && rank_sum[tid]) atomicAdd(&splits_acc[s * R + tid], rank_sum[tid]);
         uint16_t* out_rank = in_rank + (size_t)t0 * K;
         for (int a = tid; a < na; a += kLThreads) {
             const int e = eidx[a];
@@ -262,34 +332,30 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
     const int nrows = E + R;
 
     if (coop) {
-        // ---------------------- cooperative: phase 2 over the whole grid ---
+        // ------- cooperative: one barrier, then phase 3 and phase 2 at once ---
         if (!grid_barrier(counter, gridDim.x)) {
             if (tid == 0) atomicOr(status, MOE_ST_TIMEOUT);
             return;
         }
-        for (int p = j * kLWarps + warp; p < nrows; p += gridDim.x * kLWarps) {
-            const RowOut o = scan_row(p, E, R, geo, tile_base, tile_tpr, nullptr, bs, counts,
-                                      tokens_per_rank);
-            if (p < E && lane == 0) {
-                tokens_per_expert[p] = o.total;
-                expert_count[p] = o.total;
+        const int G = gridDim.x;
+        if (j == 0) {
+            if (tid < E) {
+                const int c = __ldcg(expert_count + tid);
+                tokens_per_expert[tid] = c;
+                ctot[tid] = ((c + align - 1) / align) * align;
             }
+            for (int q = tid; q < R * R; q += kLThreads) splits[q] = __ldcg(splits_acc + q);
+            __syncthreads();
+            const int total = block_exclusive_scan_1024(ctot, E, scratch);
+            if (tid < E) offsets[tid] = ctot[tid];
+            if (tid == 0) offsets[E] = total;
+            if (G > 1) return;
         }
-        if (!grid_barrier(counter, 2u * gridDim.x)) {
-            if (tid == 0) atomicOr(status, MOE_ST_TIMEOUT);
-            return;
-        }
-        if (j != 0) return;
-        // phase 3 inputs from global memory
-        for (int q = tid; q < R * R; q += kLThreads) acc_splits[q] = 0;
-        if (tid < E) ctot[tid] = __ldcg(expert_count + tid);
-        __syncthreads();
-        const int n = R * E;
-        for (int q = tid; q < n; q += kLThreads) {
-            const int v = __ldcg(counts + q);
-            if (v) atomicAdd(&acc_splits[q / El], v);
-        }
-        __syncthreads();
+        const int row_ctas = G > 1 ? G - 1 : 1;
+        const int cta_rank = G > 1 ? j - 1 : 0;
+        for (int p = cta_rank * kLWarps + warp; p < nrows; p += row_ctas * kLWarps)
+            scan_row_regs(p, E, R, geo, tile_base, tile_tpr, bs, counts, tokens_per_rank);
+        return;
     } else {
         // ------------------- the last CTA to arrive runs phases 2 and 3 ---
         __threadfence();
@@ -365,13 +431,13 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
         if (e != cudaSuccess) return e;
         configured[dev] = (int)smem;
     }
-    // Zero the arrival counter, then one launch: cooperative (grid barriers)
-    // when one CTA per tile fits on the GPU at once, else last-CTA.
-    LayoutHeader* hdr = reinterpret_cast<LayoutHeader*>(ws);
-    cudaError_t err = cudaMemsetAsync(&hdr->done, 0, sizeof(hdr->done), stream);
+    // Zero the arrival counter and the accumulators, then one launch:
+    // cooperative (one grid barrier) when one CTA per tile fits on the GPU at
+    // once, else last-CTA.
+    cudaError_t err = cudaMemsetAsync(ws + wl.zero_begin, 0, wl.zero_end - wl.zero_begin, stream);
     if (err != cudaSuccess) return err;
     const int grid = geo.n_tiles > 0 ? geo.n_tiles : 1;
-    int coop = grid <= sm_count_current_device() ? 1 : 0;
+    int coop = (grid <= sm_count_current_device() && grid <= kCoopMaxTiles) ? 1 : 0;
     if (coop) {
         static int coop_ok[64] = {};
         if (dev >= 0 && dev < 64 && coop_ok[dev] == 0) {
@@ -381,7 +447,7 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
         }
         if (dev < 0 || dev >= 64 || coop_ok[dev] != 1) coop = 0;
     }
-    // With barriers, phase 2 reads the rows from global memory: no staging.
+    // With the barrier, phase 2 reads the rows from global memory: no staging.
     const int stg = coop ? 0 : staged;
     if (coop) {
         void* args[] = {(void*)&topk_idx, (void*)&T, (void*)&K, (void*)&E, (void*)&R,

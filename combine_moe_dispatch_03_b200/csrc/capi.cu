@@ -1,7 +1,11 @@
 // capi.cu -- the extern "C" entry points of libmoe_dispatch.so: argument
 // checks on the host, then kernel launches on the caller's stream.  No call
-// allocates, synchronises or reads device memory on the host.
+// allocates, synchronises or reads device memory on the host.  Every call
+// that enqueues work is an NVTX range named after the call, so a profiler
+// timeline shows which kernels each call launched (header-only NVTX: without
+// a tool attached a range costs a branch).
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 
@@ -47,6 +51,13 @@ bool ncap_ok(int64_t N_cap, int T, int K) {
 
 int finish(cudaError_t err) { return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 }  // namespace
 
 extern "C" {
@@ -67,6 +78,7 @@ int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int
                         int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
                         int32_t* expert_offsets, void* workspace, int32_t* status,
                         cudaStream_t stream) {
+    NvtxRange range("moe_dispatch_layout");
     if (!sizes_ok(T, K, E) || R < 1 || R > MOE_MAX_R || E % R || T % R || align < 1)
         return MOE_ERR_INVALID_ARG;
     if ((int64_t)T * K + (int64_t)E * (align - 1) > INT32_MAX) return MOE_ERR_INVALID_ARG;
@@ -87,6 +99,7 @@ int moe_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E,
                 const int32_t* expert_offsets, const void* workspace, int zero_pad,
                 int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat, int32_t* flat_to_row,
                 int32_t* status, cudaStream_t stream) {
+    NvtxRange range("moe_permute");
     if (!sizes_ok(T, K, E) || !hidden_ok(H) || !ncap_ok(N_cap, T, K)) return MOE_ERR_INVALID_ARG;
     if (!expert_offsets || !workspace || !status) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !topk_idx || !flat_to_row)) return MOE_ERR_INVALID_ARG;
@@ -103,6 +116,7 @@ int moe_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E,
 int moe_expert_scale(const uint16_t* rows, int64_t N_cap, const int32_t* expert_offsets,
                      const int32_t* tokens_per_expert, int E, int H, const float* scales,
                      uint16_t* out, int32_t* status, cudaStream_t stream) {
+    NvtxRange range("moe_expert_scale");
     if (E < 1 || E > MOE_MAX_E || !hidden_ok(H) || N_cap < 0 || N_cap > INT32_MAX)
         return MOE_ERR_INVALID_ARG;
     if (!expert_offsets || !tokens_per_expert || !scales || !status) return MOE_ERR_INVALID_ARG;
@@ -119,6 +133,7 @@ int moe_combine_weighted(const uint16_t* rows, int64_t N_cap, const int32_t* row
                          const int32_t* flat_to_row, const void* weights, int weight_dtype,
                          int T, int K, int H, int validate, uint16_t* out, int32_t* status,
                          cudaStream_t stream) {
+    NvtxRange range("moe_combine_weighted");
     if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || !hidden_ok(H) ||
         N_cap < 0 || N_cap > INT32_MAX)
         return MOE_ERR_INVALID_ARG;
@@ -142,6 +157,7 @@ int moe_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t
                          const int32_t* expert_offsets, int E, int zero_pad,
                          uint16_t* grad_rows, void* grad_weights, int32_t* status,
                          cudaStream_t stream) {
+    NvtxRange range("moe_combine_backward");
     if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || !hidden_ok(H) ||
         N_cap < 0 || N_cap > INT32_MAX || E < 1 || E > MOE_MAX_E)
         return MOE_ERR_INVALID_ARG;
@@ -166,6 +182,7 @@ int moe_permute_payload(const void* x, int64_t row_bytes, const void* aux, int64
                         const int32_t* expert_offsets, const void* workspace, int zero_pad,
                         int64_t N_cap, void* x_perm, void* aux_perm, int32_t* row_to_flat,
                         int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
+    NvtxRange range("moe_permute_payload");
     if (!sizes_ok(T, K, E) || !ncap_ok(N_cap, T, K)) return MOE_ERR_INVALID_ARG;
     if (row_bytes <= 0 || row_bytes % 16 || row_bytes / 16 > INT32_MAX / 2) return MOE_ERR_INVALID_ARG;
     if (aux_row_bytes < 0 || aux_row_bytes % 4 || aux_row_bytes > 65536) return MOE_ERR_INVALID_ARG;
@@ -186,6 +203,7 @@ int moe_combine_weighted_f32(const float* rows, int64_t N_cap, const int32_t* ro
                              const int32_t* flat_to_row, const void* weights, int weight_dtype,
                              int T, int K, int H, int validate, float* out, int32_t* status,
                              cudaStream_t stream) {
+    NvtxRange range("moe_combine_weighted_f32");
     if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || H <= 0 || H % 4 ||
         N_cap < 0 || N_cap > INT32_MAX)
         return MOE_ERR_INVALID_ARG;
@@ -209,6 +227,7 @@ int moe_combine_backward_f32(const float* grad_out, const float* rows, int64_t N
                              const int32_t* expert_offsets, int E, int zero_pad,
                              float* grad_rows, void* grad_weights, int32_t* status,
                              cudaStream_t stream) {
+    NvtxRange range("moe_combine_backward_f32");
     if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || H <= 0 || H % 4 ||
         N_cap < 0 || N_cap > INT32_MAX || E < 1 || E > MOE_MAX_E)
         return MOE_ERR_INVALID_ARG;
@@ -231,6 +250,7 @@ int moe_combine_backward_f32(const float* grad_out, const float* rows, int64_t N
 
 int moe_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
                            int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
+    NvtxRange range("moe_scatter_flat_index");
     if (T < 0 || K < 1 || K > MOE_MAX_K || (int64_t)T * K > INT32_MAX || N < 0 || N > INT32_MAX)
         return MOE_ERR_INVALID_ARG;
     if (!status || (N > 0 && !row_flat) || (T > 0 && !flat_to_row)) return MOE_ERR_INVALID_ARG;

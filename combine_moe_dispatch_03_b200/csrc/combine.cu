@@ -61,6 +61,8 @@ combine_kernel(const uint4* __restrict__ rows, int64_t N_cap, const int32_t* __r
                const int32_t* __restrict__ f2r, const void* __restrict__ w, int wdtype, int T,
                int K, int n16, uint4* __restrict__ out, int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    pdl_wait();
+    pdl_trigger();
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     int bad = 0;
 
@@ -147,6 +149,8 @@ combine_slots_kernel(const uint4* __restrict__ rows, int64_t N_cap,
                      const void* __restrict__ w, int wdtype, int T, int n16,
                      uint4* __restrict__ out, int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    pdl_wait();
+    pdl_trigger();
     const int chunks = (n16 + 32 * U - 1) / (32 * U);
     const int64_t n_items = (int64_t)T * chunks;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
@@ -241,6 +245,8 @@ combine_bwd_kernel(const uint4* __restrict__ g, const uint4* __restrict__ rows,
                    uint4* __restrict__ grad_rows, void* __restrict__ grad_w,
                    int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    pdl_wait();
+    pdl_trigger();
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     int bad = 0;
 
@@ -335,6 +341,8 @@ combine_bwd_slots_kernel(const uint4* __restrict__ g, const uint4* __restrict__ 
                          uint4* __restrict__ grad_rows, void* __restrict__ grad_w,
                          int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    pdl_wait();
+    pdl_trigger();
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     int bad = 0;
 
@@ -449,8 +457,8 @@ template <typename Tr, bool V>
 static void launch_combine_t(int K, int grid, cudaStream_t st, const uint4* rows, int64_t N_cap,
                              const int32_t* r2f, const int32_t* f2r, const void* w, int wd, int T,
                              int n16, uint4* out, int32_t* status) {
-    combine_kernel<Tr, 2, V><<<grid, kBlock, 0, st>>>(rows, N_cap, r2f, f2r, w, wd, T, K, n16, out,
-                                                      status);
+    launch_pdl(combine_kernel<Tr, 2, V>, dim3(grid), dim3(kBlock), 0, st, rows, N_cap, r2f, f2r, w,
+               wd, T, K, n16, out, status);
 }
 
 // Enough warps for one token each (up to 8 resident CTAs per SM), and, when a
@@ -478,14 +486,14 @@ static void launch_slots_t(int K, int grid, cudaStream_t st, const uint4* rows, 
     constexpr int U = MOE_COMBINE_U, D = MOE_COMBINE_D;
     // Small K: wider chunks keep as many vectors in flight per lane.
     switch (K) {
-        case 1: combine_slots_kernel<Tr, 1, 4 * U, 1, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
-        case 2: combine_slots_kernel<Tr, 2, 2 * U, 2, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
-        case 3: combine_slots_kernel<Tr, 3, U, (D < 3 ? D : 3), V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
-        case 4: combine_slots_kernel<Tr, 4, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
-        case 5: combine_slots_kernel<Tr, 5, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
-        case 6: combine_slots_kernel<Tr, 6, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
-        case 7: combine_slots_kernel<Tr, 7, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
-        default: combine_slots_kernel<Tr, 8, U, D, V><<<grid, kBlock, 0, st>>>(MOE_SLOTS_ARGS); break;
+        case 1: launch_pdl(combine_slots_kernel<Tr, 1, 4 * U, 1, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 2: launch_pdl(combine_slots_kernel<Tr, 2, 2 * U, 2, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 3: launch_pdl(combine_slots_kernel<Tr, 3, U, (D < 3 ? D : 3), V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 4: launch_pdl(combine_slots_kernel<Tr, 4, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 5: launch_pdl(combine_slots_kernel<Tr, 5, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 6: launch_pdl(combine_slots_kernel<Tr, 6, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 7: launch_pdl(combine_slots_kernel<Tr, 7, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        default: launch_pdl(combine_slots_kernel<Tr, 8, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
     }
 }
 
@@ -562,18 +570,17 @@ static cudaError_t launch_backward_rows(const uint4* g, const uint4* rows, int64
 #endif
     constexpr int U = MOE_BWD_U, D = MOE_BWD_D;
     switch (K) {
-        case 1: combine_bwd_slots_kernel<Tr, 1, 4 * U, 1><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 2: combine_bwd_slots_kernel<Tr, 2, 2 * U, 2><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 3: combine_bwd_slots_kernel<Tr, 3, U, (D < 3 ? D : 3)><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 4: combine_bwd_slots_kernel<Tr, 4, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 5: combine_bwd_slots_kernel<Tr, 5, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 6: combine_bwd_slots_kernel<Tr, 6, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 7: combine_bwd_slots_kernel<Tr, 7, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
-        case 8: combine_bwd_slots_kernel<Tr, 8, U, D><<<grid, kBlock, 0, stream>>>(MOE_BWD_SLOT_ARGS); break;
+        case 1: launch_pdl(combine_bwd_slots_kernel<Tr, 1, 4 * U, 1>, dim3(grid), dim3(kBlock), 0, stream, MOE_BWD_SLOT_ARGS); break;
+        case 2: launch_pdl(combine_bwd_slots_kernel<Tr, 2, 2 * U, 2>, dim3(grid), dim3(kBlock), 0, stream, MOE_BWD_SLOT_ARGS); break;
+        case 3: launch_pdl(combine_bwd_slots_kernel<Tr, 3, U, (D < 3 ? D : 3)>, dim3(grid), dim3(kBlock), 0, stream, MOE_BWD_SLOT_ARGS); break;
+        case 4: launch_pdl(combine_bwd_slots_kernel<Tr, 4, U, D>, dim3(grid), dim3(kBlock), 0, stream, MOE_BWD_SLOT_ARGS); break;
+        case 5: launch_pdl(combine_bwd_slots_kernel<Tr, 5, U, D>, dim3(grid), dim3(kBlock), 0, stream, MOE_BWD_SLOT_ARGS); break;
+        case 6: launch_pdl(combine_bwd_slots_kernel<Tr, 6, U, D>, dim3(grid), dim3(kBlock), 0, stream, MOE_BWD_SLOT_ARGS); break;
+        case 7: launch_pdl(combine_bwd_slots_kernel<Tr, 7, U, D>, dim3(grid), dim3(kBlock), 0, stream, MOE_BWD_SLOT_ARGS); break;
+        case 8: launch_pdl(combine_bwd_slots_kernel<Tr, 8, U, D>, dim3(grid), dim3(kBlock), 0, stream, MOE_BWD_SLOT_ARGS); break;
         default:
-            combine_bwd_kernel<Tr><<<grid, kBlock, 0, stream>>>(g, rows, N_cap, r2f, f2r, w, wd, T,
-                                                                K, n16, offsets, E, zero_pad,
-                                                                grad_rows, grad_w, status);
+            launch_pdl(combine_bwd_kernel<Tr>, dim3(grid), dim3(kBlock), 0, stream, g, rows, N_cap, r2f,
+                       f2r, w, wd, T, K, n16, offsets, E, zero_pad, grad_rows, grad_w, status);
             break;
     }
     return cudaGetLastError();

@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moe_dispatch.h"
 
 namespace moe {
@@ -17,6 +19,42 @@ namespace moe {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kBlock = 256;               // threads per CTA for every kernel
 constexpr int kWarps = kBlock / 32;
+
+// --------------------------------------------- programmatic dependent launch ---
+//
+// The streaming kernels are launched with programmatic stream serialization
+// (launch_pdl): the next kernel on the stream may be scheduled onto SMs while
+// this one drains, instead of after it has fully retired.  Every such kernel
+// calls pdl_wait() before its first global-memory access: it returns once the
+// preceding kernel on the stream has completed and its writes are visible,
+// so the ordering the caller sees is exactly stream order.  pdl_trigger()
+// (after the wait) lets the following kernel be scheduled as soon as every
+// CTA of this grid has started.  After a non-kernel operation (memset, event,
+// copy) or a kernel that never triggers, both are plain stream order.
+#ifndef MOE_PDL
+#define MOE_PDL 1
+#endif
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = MOE_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------ bf16 ---
 

@@ -29,6 +29,8 @@ expert_scale_kernel(const uint16_t* __restrict__ rows, int64_t N_cap,
     int* cnt = off + (E + 1);                      // [E]
     float* sc = reinterpret_cast<float*>(cnt + E); // [E]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    pdl_trigger();
     for (int e = tid; e <= E; e += kBlock) off[e] = offsets[e];
     for (int e = tid; e < E; e += kBlock) {
         cnt[e] = counts[e];
@@ -82,10 +84,8 @@ cudaError_t launch_expert_scale(const uint16_t* rows, int64_t N_cap, const int32
     if (want < grid) grid = (int)want;
     if (grid < 1) grid = 1;
     const size_t smem = sizeof(int) * (2 * (size_t)E + 1) + sizeof(float) * (size_t)E;
-    expert_scale_kernel<MOE_SCALE_U><<<grid, kBlock, smem, stream>>>(rows, N_cap, expert_offsets,
-                                                           tokens_per_expert, E, H, scales, out,
-                                                           status);
-    return cudaGetLastError();
+    return launch_pdl(expert_scale_kernel<MOE_SCALE_U>, dim3(grid), dim3(kBlock), smem, stream,
+                      rows, N_cap, expert_offsets, tokens_per_expert, E, H, scales, out, status);
 }
 
 }  // namespace moe

@@ -41,6 +41,8 @@ permute_kernel(const uint4* __restrict__ x, int n16, const uint32_t* __restrict_
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int scratch[kWarps + 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    pdl_trigger();
     const LayoutHeader* hdr = reinterpret_cast<const LayoutHeader*>(ws);
     if (hdr->magic != kLayoutMagic || hdr->T != T || hdr->K != K || hdr->E != E) {
         if (blockIdx.x == 0 && tid == 0) atomicOr(status, MOE_ST_LAYOUT_MISMATCH);
@@ -159,11 +161,10 @@ static cudaError_t launch_rows(const uint4* x, int n16, const uint32_t* aux, int
 #endif
     if (grid > (int64_t)sms * MOE_PERMUTE_GRID_PER_SM) grid = (int64_t)sms * MOE_PERMUTE_GRID_PER_SM;
     if (grid < 1) grid = 1;
-    permute_kernel<U, AUX><<<(int)grid, kBlock, sizeof(int) * 2 * ((size_t)E + 1), stream>>>(
-        x, n16, aux, aux_words, topk_idx, T, K, E, expert_offsets,
-        static_cast<const char*>(workspace), zero_pad, N_cap, x_perm, aux_perm, row_to_flat,
-        flat_to_row, status);
-    return cudaGetLastError();
+    return launch_pdl(permute_kernel<U, AUX>, dim3((int)grid), dim3(kBlock),
+                      sizeof(int) * 2 * ((size_t)E + 1), stream, x, n16, aux, aux_words, topk_idx,
+                      T, K, E, expert_offsets, static_cast<const char*>(workspace), zero_pad,
+                      N_cap, x_perm, aux_perm, row_to_flat, flat_to_row, status);
 }
 
 cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,

@@ -11,7 +11,8 @@ import pytest
 import torch
 
 from _pipeline import SENTINEL, compare, run_gpu, run_oracle
-from combine_moe_dispatch_03_b200.inputs import CONFIGS, capacity_rows, custom_inputs, make_inputs
+from combine_moe_dispatch_03_b200.inputs import (CONFIGS, bf16_bits, capacity_rows, custom_inputs,
+                                                 make_inputs)
 
 pytestmark = pytest.mark.gpu
 
@@ -151,3 +152,37 @@ def test_combine_token_chunks_concatenate():
     a = api.combine_weighted(xp, f2r[:h].contiguous(), w[:h].contiguous())
     b = api.combine_weighted(xp, f2r[h:].contiguous(), w[h:].contiguous())
     assert torch.equal(full.view(torch.int16), torch.cat([a, b]).view(torch.int16))
+
+
+def test_layout_workspace_reused_across_calls():
+    """One workspace, never initialised by the caller, serves several layouts
+    in a row: each call's counts, offsets and rows match the oracle, whatever
+    the previous call (or garbage) left in it."""
+    import oracle as orc
+    from combine_moe_dispatch_03_b200 import api
+    dev = torch.device("cuda:0")
+    T, H, E, K, R, align = 2048, 64, 128, 8, 8, 16
+    lay = api.alloc_layout(T, K, E, R, align, dev)
+    lay.workspace.fill_(0xA5)                               # garbage, as from a caching allocator
+    N = capacity_rows(T, K, E, align)
+    g = torch.Generator().manual_seed(77)
+    routings = [torch.randint(0, E, (T, K), generator=g),
+                torch.randint(0, 5, (T, K), generator=g),     # heavy skew, repeats in a token
+                None]
+    routings[2] = routings[0]
+    for topk in routings:
+        inp = custom_inputs(T, H, E, K, seed=3, topk_idx=topk)
+        st = api.new_status(dev)
+        api.dispatch_layout(inp["topk_idx"].to(dev), E, R, align, status=st, out=lay)
+        xp, r2f, f2r = api.permute(inp["x"].to(dev), inp["topk_idx"].to(dev), lay, capacity=N,
+                                   status=st)
+        api.check_status(st)
+        ref = orc.layout(inp["topk_idx"].numpy(), E, R, align)
+        for key in ("tokens_per_expert", "counts", "splits", "tokens_per_rank", "is_token_in_rank",
+                    "expert_offsets"):
+            np.testing.assert_array_equal(getattr(lay, key).cpu().numpy(), ref[key], err_msg=key)
+        pm = orc.permute(bf16_bits(inp["x"]), inp["topk_idx"].numpy(), E, ref["expert_offsets"], N)
+        np.testing.assert_array_equal(f2r.cpu().numpy(), pm["flat_to_row"])
+        np.testing.assert_array_equal(r2f.cpu().numpy(), pm["row_to_flat"])
+        n_pad = int(ref["expert_offsets"][-1])                # rows past it are left untouched
+        np.testing.assert_array_equal(bf16_bits(xp[:n_pad].cpu()), pm["x_perm"][:n_pad])

@@ -76,3 +76,37 @@ def test_forward_makes_no_host_sync():
         torch.cuda.set_sync_debug_mode("default")
     torch.cuda.synchronize()
     assert int(status.item()) == 0
+
+
+def test_split_dispatch_combine_with_a_torch_expert():
+    """dispatch / combine as separate autograd Functions with the caller's
+    own expert in between (here y = 2 * x_perm in torch, exact in bf16):
+    output and both gradients equal, bit for bit, the chain with the
+    stand-in expert at s_e = 2, whose gradients the oracle pins above."""
+    from combine_moe_dispatch_03_b200 import api
+    from combine_moe_dispatch_03_b200.autograd import combine, dispatch, moe_dispatch_combine
+    cfg = CONFIGS["qwen3"]
+    inp = make_inputs("qwen3", T=2048, with_grad=True)
+    dev = torch.device("cuda:0")
+    topk = inp["topk_idx"].to(dev)
+    g = inp["grad_out"].to(dev)
+    two = torch.full((cfg.E,), 2.0, dtype=torch.float32, device=dev)
+
+    x1 = inp["x"].to(dev).requires_grad_(True)
+    w1 = inp["weights"].to(dev).requires_grad_(True)
+    out1, st1 = moe_dispatch_combine(x1, topk, w1, two, cfg.E, cfg.R, cfg.align)
+    out1.backward(g)
+
+    x2 = inp["x"].to(dev).requires_grad_(True)
+    w2 = inp["weights"].to(dev).requires_grad_(True)
+    x_perm, handle = dispatch(x2, topk, cfg.E, cfg.R, cfg.align)
+    out2 = combine(x_perm * 2, handle, w2, validate=True)
+    out2.backward(g)
+    api.check_status(st1)
+    api.check_status(handle.status)
+
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(x1.grad.view(torch.int16), x2.grad.view(torch.int16))
+    assert torch.equal(w1.grad, w2.grad)
+    off = handle.layout.expert_offsets
+    assert int(off[-1]) <= handle.num_rows

@@ -31,6 +31,8 @@
 //
 // Bytes: reads topk_idx once (8*A), writes the [T,R] flags, in-tile ranks
 // (2*A) and O((E+R) * tiles) ints.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -422,14 +424,21 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
     const int staged = (p2 + stage) <= kLayoutSmemMax ? 1 : 0;
     const size_t p2s = p2 + (staged ? stage : 0);
     const size_t smem = p1 > p2s ? p1 : p2s;
-    static int configured[64] = {};
+    // Per-device caches (host threads may call concurrently: atomics).
+    static std::atomic<int> configured[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-    if (smem > 48 * 1024 && dev >= 0 && dev < 64 && configured[dev] < (int)smem) {
+    if (smem > 48 * 1024 &&
+        (dev < 0 || dev >= 64 || configured[dev].load(std::memory_order_relaxed) < (int)smem)) {
         const cudaError_t e = cudaFuncSetAttribute(
             layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        configured[dev] = (int)smem;
+        if (dev >= 0 && dev < 64) {
+            int cur = configured[dev].load(std::memory_order_relaxed);
+            while (cur < (int)smem &&
+                   !configured[dev].compare_exchange_weak(cur, (int)smem, std::memory_order_relaxed)) {
+            }
+        }
     }
     // Zero the arrival counter and the accumulators, then one launch:
     // cooperative (one grid barrier) when one CTA per tile fits on the GPU at
@@ -439,13 +448,14 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
     const int grid = geo.n_tiles > 0 ? geo.n_tiles : 1;
     int coop = (grid <= sm_count_current_device() && grid <= kCoopMaxTiles) ? 1 : 0;
     if (coop) {
-        static int coop_ok[64] = {};
-        if (dev >= 0 && dev < 64 && coop_ok[dev] == 0) {
+        static std::atomic<int> coop_ok[64];
+        if (dev >= 0 && dev < 64 && coop_ok[dev].load(std::memory_order_relaxed) == 0) {
             int attr = 0;
-            cudaDeviceGetAttribute(&attr, cudaDevAttrCooperativeLaunch, dev);
-            coop_ok[dev] = attr ? 1 : -1;
+            if (cudaDeviceGetAttribute(&attr, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess)
+                attr = 0;
+            coop_ok[dev].store(attr ? 1 : -1, std::memory_order_relaxed);
         }
-        if (dev < 0 || dev >= 64 || coop_ok[dev] != 1) coop = 0;
+        if (dev < 0 || dev >= 64 || coop_ok[dev].load(std::memory_order_relaxed) != 1) coop = 0;
     }
     // With the barrier, phase 2 reads the rows from global memory: no staging.
     const int stg = coop ? 0 : staged;

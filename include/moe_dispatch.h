@@ -38,10 +38,14 @@
  *  - Every data pointer is caller-owned DEVICE memory of the current device.
  *    The library allocates nothing and never synchronises with the host;
  *    every call only enqueues work on `stream` (a cudaStream_t; NULL is the
- *    legacy default stream) and returns: kernels, plus for the layout a
- *    4-byte memset of its workspace counter.  Results are defined once the
- *    stream reaches them.  The only state kept between calls is a per-device
- *    cache of the SM count.
+ *    legacy default stream) and returns: kernels, plus for the layout one
+ *    memset of its workspace counter and accumulators (4 + 4E + 4R*R bytes).
+ *    Results are defined once the stream reaches them.  The streaming
+ *    kernels use programmatic dependent launch: each waits for the kernel
+ *    before it on the stream to complete before its first memory access, so
+ *    the order the caller sees is plain stream order.  The only state kept
+ *    between calls is per-device caches of launch attributes (SM count,
+ *    cooperative-launch support, the layout's shared-memory opt-in).
  *  - Notation: T tokens, H hidden size (bf16 elements per row), E experts,
  *    K = top_k, R logical ranks, El = E/R, align = group alignment,
  *    A = T*K assignments, flat index f = t*K + k (token t, slot k),
@@ -134,10 +138,11 @@ int64_t moe_worst_case_rows(int T, int K, int E, int align);
  *                                     takes no rows)
  *      workspace                      moe_layout_workspace_bytes(T,K,E,R)
  *                                     bytes, 16-byte aligned
- * Launch: one kernel of about one 1024-thread CTA per SM, cooperative (its
- * phases are separated by grid barriers) when all its CTAs fit on the GPU at
- * once; a barrier that does not complete within 2 s gives up and sets
- * MOE_ST_TIMEOUT.
+ * Launch: a memset of the workspace's counter and accumulators, then one
+ * kernel of about one 1024-thread CTA per SM, cooperative (its tile ranking
+ * and its scans are separated by one grid barrier) when all its CTAs fit on
+ * the GPU at once; a barrier that does not complete within 2 s gives up and
+ * sets MOE_ST_TIMEOUT.
  * Status: MOE_ST_EXPERT_OOR (that assignment is left out of every count),
  *         MOE_ST_TIMEOUT.
  * Errors: MOE_ERR_INVALID_ARG for a null pointer, sizes outside the limits,
@@ -166,8 +171,10 @@ int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int
  *  - The first call on a device looks up the array's device address (with
  *    that device current) and caches it; make that first call before any
  *    stream capture on the device.
- *  - Every call shares the one array, which keeps the last call's contents
- *    (the kernels rewrite every word they read, so nothing needs clearing).
+ *  - Every call shares the one array, which keeps the last call's contents;
+ *    the call clears what must start at zero (a memset of the layout's
+ *    counter and accumulators, enqueued on `stream`) and its kernel rewrites
+ *    every other word it reads, so the caller clears nothing.
  *    Calls that overlap on the GPU -- on different streams, or from threads
  *    whose streams are not ordered -- race on it and give undefined results.
  *  - The permute cannot use this scratch; a caller that also permutes uses

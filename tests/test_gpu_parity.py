@@ -186,3 +186,20 @@ def test_layout_workspace_reused_across_calls():
         np.testing.assert_array_equal(r2f.cpu().numpy(), pm["row_to_flat"])
         n_pad = int(ref["expert_offsets"][-1])                # rows past it are left untouched
         np.testing.assert_array_equal(bf16_bits(xp[:n_pad].cpu()), pm["x_perm"][:n_pad])
+
+
+def test_side_stream_matches_default_stream():
+    """Every call enqueues on the caller's current stream: the whole chain
+    run on a side stream (kernels back to back, no host sync in between)
+    gives the same bytes as on the default stream."""
+    cfg = CONFIGS["qwen3"]
+    inp = make_inputs("qwen3", T=2048, with_grad=True)
+    N = capacity_rows(2048, cfg.K, cfg.E, cfg.align)
+    a = run_gpu(inp, cfg.E, cfg.R, cfg.align, N)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        b = run_gpu(inp, cfg.E, cfg.R, cfg.align, N)
+    for k in ("expert_offsets", "counts", "x_perm", "row_to_flat", "flat_to_row", "y", "out",
+              "grad_rows", "grad_w", "grad_x"):
+        np.testing.assert_array_equal(a[k], b[k], err_msg=k)

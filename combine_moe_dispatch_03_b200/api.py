@@ -45,6 +45,24 @@ def _require(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int | None = 
         raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
 
 
+def _check_out(t: torch.Tensor, name: str, shape: tuple, dtype: torch.dtype, device):
+    """A caller-provided output (or a tensor whose size another fixes): the
+    kernels write/read exactly `shape`, so anything else is refused here,
+    before any launch."""
+    _require(t, name, dtype)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _check_layout(layout: "Layout", T: int, K: int, device):
+    if layout.T != T or layout.K != K:
+        raise ValueError(f"layout was built for T={layout.T}, K={layout.K}; got T={T}, K={K}")
+    if layout.expert_offsets.device != device:
+        raise ValueError(f"layout is on {layout.expert_offsets.device}, expected {device}")
+
+
 def _weight_dtype(w: torch.Tensor) -> int:
     if w.dtype == torch.float32:
         return DTYPE_F32
@@ -115,6 +133,11 @@ def dispatch_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int = 1
     _require(topk_idx, "topk_idx", torch.int64, 2)
     T, K = topk_idx.shape
     dev = topk_idx.device
+    if out is not None and (out.T, out.K, out.E, out.R) != (T, K, num_experts, num_ranks):
+        raise ValueError(f"out layout was allocated for (T, K, E, R) = {(out.T, out.K, out.E, out.R)}, "
+                         f"got {(T, K, num_experts, num_ranks)}")
+    if out is not None:
+        out.align = align
     lay = out if out is not None else alloc_layout(T, K, num_experts, num_ranks, align, dev)
     st = status if status is not None else new_status(dev)
     rc = lib().moe_dispatch_layout(
@@ -134,6 +157,8 @@ def permute(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout, capacity: i
     T, H = x.shape
     K = topk_idx.shape[1]
     dev = x.device
+    _check_out(topk_idx, "topk_idx", (T, K), torch.int64, dev)
+    _check_layout(layout, T, K, dev)
     N_cap = capacity if capacity is not None else worst_case_rows(T, K, layout.E, layout.align)
     if out is None:
         x_perm = torch.empty(N_cap, H, dtype=torch.bfloat16, device=dev)
@@ -141,6 +166,9 @@ def permute(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout, capacity: i
         f2r = torch.empty(T, K, dtype=torch.int32, device=dev)
     else:
         x_perm, r2f, f2r = out
+        _check_out(x_perm, "x_perm", (N_cap, H), torch.bfloat16, dev)
+        _check_out(r2f, "row_to_flat", (N_cap,), torch.int32, dev)
+        _check_out(f2r, "flat_to_row", (T, K), torch.int32, dev)
     st = status if status is not None else new_status(dev)
     rc = lib().moe_permute(_ptr(x), _ptr(topk_idx), T, K, layout.E, H, _ptr(layout.expert_offsets),
                            _ptr(layout.workspace), int(bool(zero_pad)), N_cap, _ptr(x_perm),
@@ -155,7 +183,11 @@ def expert_scale(rows: torch.Tensor, layout: Layout, scales: torch.Tensor,
     _require(rows, "rows", torch.bfloat16, 2)
     _require(scales, "scales", torch.float32, 1)
     N_cap, H = rows.shape
+    _check_out(scales, "scales", (layout.E,), torch.float32, rows.device)
+    if layout.expert_offsets.device != rows.device:
+        raise ValueError("layout and rows are on different devices")
     y = out if out is not None else torch.empty_like(rows)
+    _check_out(y, "out", (N_cap, H), torch.bfloat16, rows.device)
     st = status if status is not None else new_status(rows.device)
     rc = lib().moe_expert_scale(_ptr(rows), N_cap, _ptr(layout.expert_offsets),
                                 _ptr(layout.tokens_per_expert), layout.E, H, _ptr(scales), _ptr(y),
@@ -186,8 +218,11 @@ def combine_weighted(rows: torch.Tensor, flat_to_row: torch.Tensor,
     if validate:
         if row_to_flat is None:
             raise ValueError("validate=True needs row_to_flat")
-        _require(row_to_flat, "row_to_flat", torch.int32, 1)
+        _check_out(row_to_flat, "row_to_flat", (N_cap,), torch.int32, rows.device)
+    if flat_to_row.device != rows.device or (weights is not None and weights.device != rows.device):
+        raise ValueError("rows, flat_to_row and weights must be on one device")
     o = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=rows.device)
+    _check_out(o, "out", (T, H), torch.bfloat16, rows.device)
     st = status if status is not None else new_status(rows.device)
     rc = lib().moe_combine_weighted(_ptr(rows), N_cap, _ptr(row_to_flat), _ptr(flat_to_row),
                                     _ptr(weights), wd, T, K, H, int(bool(validate)), _ptr(o),
@@ -213,11 +248,21 @@ def combine_backward(grad_out: torch.Tensor, rows: torch.Tensor, row_to_flat: to
     _require(weights, "weights", weights.dtype, 2)
     N_cap, H = rows.shape
     T, K = flat_to_row.shape
+    dev = rows.device
+    _check_out(grad_out, "grad_out", (T, H), torch.bfloat16, dev)
+    _check_out(row_to_flat, "row_to_flat", (N_cap,), torch.int32, dev)
+    _check_out(weights, "weights", (T, K), weights.dtype, dev)
+    _check_out(flat_to_row, "flat_to_row", (T, K), torch.int32, dev)
+    if layout.expert_offsets.device != dev:
+        raise ValueError("layout and rows are on different devices")
     if out is None:
         grad_rows = torch.empty_like(rows)
         grad_w = torch.empty(T, K, dtype=weights.dtype, device=rows.device) if want_grad_weights else None
     else:
         grad_rows, grad_w = out
+        _check_out(grad_rows, "grad_rows", (N_cap, H), torch.bfloat16, dev)
+        if grad_w is not None:
+            _check_out(grad_w, "grad_weights", (T, K), weights.dtype, dev)
     st = status if status is not None else new_status(rows.device)
     rc = lib().moe_combine_backward(_ptr(grad_out), _ptr(rows), N_cap, _ptr(row_to_flat),
                                     _ptr(flat_to_row), _ptr(weights), wd, T, K, H,
@@ -233,6 +278,7 @@ def scatter_flat_index(row_flat: torch.Tensor, T: int, K: int,
     with the folded restore's coverage check (MOE_ST_COVERAGE)."""
     _require(row_flat, "row_flat", torch.int32, 1)
     f2r = out if out is not None else torch.empty(T, K, dtype=torch.int32, device=row_flat.device)
+    _check_out(f2r, "out", (T, K), torch.int32, row_flat.device)
     st = status if status is not None else new_status(row_flat.device)
     rc = lib().moe_scatter_flat_index(_ptr(row_flat), row_flat.shape[0], T, K, _ptr(f2r),
                                       _ptr(st), _stream(row_flat.device))
@@ -254,8 +300,11 @@ def _combine_weighted_f32(rows, flat_to_row, weights, row_to_flat, validate, sta
     if validate:
         if row_to_flat is None:
             raise ValueError("validate=True needs row_to_flat")
-        _require(row_to_flat, "row_to_flat", torch.int32, 1)
+        _check_out(row_to_flat, "row_to_flat", (N_cap,), torch.int32, rows.device)
+    if flat_to_row.device != rows.device or (weights is not None and weights.device != rows.device):
+        raise ValueError("rows, flat_to_row and weights must be on one device")
     o = out if out is not None else torch.empty(T, H, dtype=torch.float32, device=rows.device)
+    _check_out(o, "out", (T, H), torch.float32, rows.device)
     st = status if status is not None else new_status(rows.device)
     rc = lib().moe_combine_weighted_f32(_ptr(rows), N_cap, _ptr(row_to_flat), _ptr(flat_to_row),
                                         _ptr(weights), wd, T, K, H, int(bool(validate)), _ptr(o),
@@ -274,11 +323,20 @@ def _combine_backward_f32(grad_out, rows, row_to_flat, flat_to_row, weights, lay
     _require(weights, "weights", weights.dtype, 2)
     N_cap, H = rows.shape
     T, K = flat_to_row.shape
+    dev = rows.device
+    _check_out(grad_out, "grad_out", (T, H), torch.float32, dev)
+    _check_out(row_to_flat, "row_to_flat", (N_cap,), torch.int32, dev)
+    _check_out(weights, "weights", (T, K), weights.dtype, dev)
+    if layout.expert_offsets.device != dev:
+        raise ValueError("layout and rows are on different devices")
     if out is None:
         grad_rows = torch.empty_like(rows)
         grad_w = torch.empty(T, K, dtype=weights.dtype, device=rows.device) if want_grad_weights else None
     else:
         grad_rows, grad_w = out
+        _check_out(grad_rows, "grad_rows", (N_cap, H), torch.float32, dev)
+        if grad_w is not None:
+            _check_out(grad_w, "grad_weights", (T, K), weights.dtype, dev)
     st = status if status is not None else new_status(rows.device)
     rc = lib().moe_combine_backward_f32(_ptr(grad_out), _ptr(rows), N_cap, _ptr(row_to_flat),
                                         _ptr(flat_to_row), _ptr(weights), wd, T, K, H,
@@ -308,6 +366,8 @@ def permute_payload(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout,
         if not aux.is_cuda or not aux.is_contiguous() or aux.shape[0] != T:
             raise ValueError("aux must be a contiguous CUDA tensor [T, ...]")
         aux_bytes = aux.element_size() * math.prod(aux.shape[1:])
+    _check_out(topk_idx, "topk_idx", (T, K), torch.int64, dev)
+    _check_layout(layout, T, K, dev)
     N_cap = capacity if capacity is not None else worst_case_rows(T, K, layout.E, layout.align)
     if out is None:
         x_perm = torch.empty((N_cap,) + tuple(x.shape[1:]), dtype=x.dtype, device=dev)
@@ -317,6 +377,13 @@ def permute_payload(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout,
         f2r = torch.empty(T, K, dtype=torch.int32, device=dev)
     else:
         x_perm, aux_perm, r2f, f2r = out
+        _check_out(x_perm, "x_perm", (N_cap,) + tuple(x.shape[1:]), x.dtype, dev)
+        if aux is not None:
+            _check_out(aux_perm, "aux_perm", (N_cap,) + tuple(aux.shape[1:]), aux.dtype, dev)
+        _check_out(r2f, "row_to_flat", (N_cap,), torch.int32, dev)
+        _check_out(f2r, "flat_to_row", (T, K), torch.int32, dev)
+    if aux is not None and aux.device != dev:
+        raise ValueError("aux and x must be on one device")
     st = status if status is not None else new_status(dev)
     rc = lib().moe_permute_payload(_ptr(x), row_bytes, _ptr(aux), aux_bytes, _ptr(topk_idx), T, K,
                                    layout.E, _ptr(layout.expert_offsets), _ptr(layout.workspace),

@@ -167,11 +167,48 @@ def test_workspace_mismatch_writes_nothing():
     r2f = torch.full((N,), 7, dtype=torch.int32, device=dev)
     f2r = torch.full((32, 2), 7, dtype=torch.int32, device=dev)
     st = api.new_status(dev)
-    api.permute(inp2["x"].to(dev), inp2["topk_idx"].to(dev), lay, capacity=N, status=st,
-                out=(xp, r2f, f2r))
+    # Through the C ABI: the Python layer would refuse this on the host (see
+    # test_python_layer_refuses_mismatched_shapes); the device check is what
+    # guards a C caller.
+    from combine_moe_dispatch_03_b200._lib import lib
+    x2, t2 = inp2["x"].to(dev), inp2["topk_idx"].to(dev)
+    rc = lib().moe_permute(x2.data_ptr(), t2.data_ptr(), 32, 2, 8, 32,
+                           lay.expert_offsets.data_ptr(), lay.workspace.data_ptr(), 1, N,
+                           xp.data_ptr(), r2f.data_ptr(), f2r.data_ptr(), st.data_ptr(),
+                           torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
     torch.cuda.synchronize()
     assert st.item() & api._lib.ST_LAYOUT_MISMATCH
     assert bool((r2f == 7).all()) and bool((f2r == 7).all())
+
+
+def test_python_layer_refuses_mismatched_shapes():
+    """Tensors whose sizes disagree with each other or with the layout are
+    refused by the binding before anything is enqueued."""
+    api, dev, inp = _setup(64, 32, 8, 2)
+    topk = inp["topk_idx"].to(dev)
+    x = inp["x"].to(dev)
+    st = api.new_status(dev)
+    lay = api.dispatch_layout(topk, 8, 2, 4, status=st)
+    xp, r2f, f2r = api.permute(x, topk, lay, status=st)
+    w = inp["weights"].to(dev)
+    torch.cuda.synchronize()
+    with pytest.raises(ValueError):                     # topk_idx rows != x rows
+        api.permute(x[:32].contiguous(), topk, lay)
+    with pytest.raises(ValueError):                     # layout built for other T
+        api.permute(x[:32].contiguous(), topk[:32].contiguous(), lay)
+    with pytest.raises(ValueError):                     # undersized output
+        api.combine_weighted(xp, f2r, w, out=torch.empty(63, 32, dtype=torch.bfloat16,
+                                                         device=dev))
+    with pytest.raises(ValueError):                     # grad_out of the wrong size
+        api.combine_backward(torch.zeros(64, 16, dtype=torch.bfloat16, device=dev), xp, r2f,
+                             f2r, w, lay)
+    with pytest.raises(ValueError):                     # scales of the wrong length
+        api.expert_scale(xp, lay, torch.ones(7, device=dev))
+    with pytest.raises(ValueError):                     # reused layout of other sizes
+        api.dispatch_layout(topk[:32].contiguous(), 8, 2, 4, out=lay)
+    torch.cuda.synchronize()
+    assert st.item() == 0
 
 
 @pytest.mark.parametrize("case", ["H%8", "misaligned", "ncap<A", "E%R", "T%R", "K>32", "E>1024"])

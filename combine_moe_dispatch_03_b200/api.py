@@ -286,6 +286,21 @@ def scatter_flat_index(row_flat: torch.Tensor, T: int, K: int,
     return f2r
 
 
+def segment_labels(counts: torch.Tensor, modulo: int, rows: int,
+                   status: torch.Tensor | None = None, out: torch.Tensor | None = None):
+    """labels [rows] int64: row i of n consecutive segments (segment j holding
+    counts[j] rows) gets j % modulo; rows past sum(counts) get -1."""
+    _require(counts, "counts", torch.int32, 1)
+    dev = counts.device
+    lab = out if out is not None else torch.empty(rows, dtype=torch.int64, device=dev)
+    _check_out(lab, "out", (rows,), torch.int64, dev)
+    st = status if status is not None else new_status(dev)
+    rc = lib().moe_segment_labels(_ptr(counts), counts.shape[0], modulo, rows, _ptr(lab), _ptr(st),
+                                  _stream(dev))
+    check_rc(rc, "moe_segment_labels")
+    return lab
+
+
 def _combine_weighted_f32(rows, flat_to_row, weights, row_to_flat, validate, status, out):
     _require(rows, "rows", torch.float32, 2)
     _require(flat_to_row, "flat_to_row", torch.int32, 2)

@@ -259,6 +259,17 @@ int moe_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
     return finish(moe::launch_scatter_flat_index(row_flat, N, T, K, flat_to_row, status, stream));
 }
 
+int moe_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows, int64_t* labels,
+                       int32_t* status, cudaStream_t stream) {
+    NvtxRange range("moe_segment_labels");
+    if (n < 1 || n > MOE_MAX_E || modulo < 1 || rows < 0 || rows > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (!counts || !status || (rows > 0 && !labels)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(counts, 4) || !aligned(labels, 8) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    return finish(moe::launch_segment_labels(counts, n, modulo, rows, labels, status, stream));
+}
+
 const char* moe_strerror(int code) {
     switch (code) {
         case MOE_OK: return "ok";

@@ -129,6 +129,9 @@ cudaError_t launch_combine_backward_f32(const float* grad_out, const float* rows
 cudaError_t launch_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
                                       int32_t* flat_to_row, int32_t* status, cudaStream_t stream);
 
+cudaError_t launch_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows,
+                                  int64_t* labels, int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t N_cap,
                                     const int32_t* row_to_flat, const int32_t* flat_to_row,
                                     const void* weights, int weight_dtype, int T, int K, int H,

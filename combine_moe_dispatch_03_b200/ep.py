@@ -47,6 +47,14 @@ def count_matrix(tokens_per_expert: torch.Tensor, ep_size: int) -> torch.Tensor:
     return tokens_per_expert.reshape(ep_size, E // ep_size)
 
 
+def plan_from_counts(counts: torch.Tensor, received: torch.Tensor) -> SplitPlan:
+    """The plan from this rank's count matrix and the received counts (what
+    the exchange delivers): row sums of both, one device-to-host copy."""
+    both = torch.stack((counts.sum(dim=1), received.sum(dim=1))).cpu()
+    return SplitPlan(input_splits=both[0].tolist(), output_splits=both[1].tolist(),
+                     received_counts=received, tokens_per_local_expert=received.sum(dim=0))
+
+
 def split_plan(counts: torch.Tensor, group=None) -> SplitPlan:
     """One all-to-all of the count matrix, one device-to-host copy."""
     ep_size = dist.get_world_size(group)
@@ -56,9 +64,7 @@ def split_plan(counts: torch.Tensor, group=None) -> SplitPlan:
     send = counts.to(torch.int32).contiguous()
     received = torch.empty_like(send)
     dist.all_to_all_single(received.view(-1), send.view(-1), group=group)
-    both = torch.stack((send.sum(dim=1), received.sum(dim=1))).cpu()
-    return SplitPlan(input_splits=both[0].tolist(), output_splits=both[1].tolist(),
-                     received_counts=received, tokens_per_local_expert=received.sum(dim=0))
+    return plan_from_counts(send, received)
 
 
 def split_plan_from_expert_indices(topk_idx: torch.Tensor, num_experts: int, group=None,
@@ -69,3 +75,102 @@ def split_plan_from_expert_indices(topk_idx: torch.Tensor, num_experts: int, gro
     ep_size = dist.get_world_size(group)
     lay = api.dispatch_layout(topk_idx, num_experts, 1, 1, status=status)
     return split_plan(count_matrix(lay.tokens_per_expert, ep_size), group)
+
+
+# ---------------------------------------------- the payload across ranks ---
+#
+# Dispatch across ranks, as steps around the two exchanges:
+#   send side:    layout of this rank's tokens (one source block, no padding)
+#                 and permute: rows in (expert, token, slot) order, which is
+#                 (destination rank, local expert, token, slot) because a
+#                 rank's experts are contiguous -- so the permuted buffer IS
+#                 the send buffer, input_splits[r] rows for rank r in turn;
+#   exchange:     the split plan, then the rows (all-to-all-v);
+#   receive side: rows arrive source by source, each source's rows in
+#                 local-expert order; labelled with their local expert
+#                 (moe_segment_labels over received_counts) they are regrouped
+#                 by expert with a top_k = 1 layout + permute (stable: source
+#                 rank, then token -- the order the single-GPU layout gives
+#                 the same expert), padded to the grouped-GEMM alignment.
+# Combine runs the same steps backwards: a unit-weight top_k = 1 combine
+# ungroups the expert outputs into received order (an exact copy), the
+# reverse exchange returns them to their source ranks in send order, and
+# fused_weighted_restore over the send side's maps gives the output.
+
+
+@dataclasses.dataclass
+class EPHandle:
+    """What dispatch across ranks leaves for combine."""
+    send_layout: api.Layout
+    send_row_to_flat: torch.Tensor      # [A]: send row -> (token, slot) of this rank
+    send_flat_to_row: torch.Tensor      # [T_local, K]
+    plan: SplitPlan
+    recv_layout: api.Layout             # received rows by local expert (top_k = 1)
+    recv_row_to_flat: torch.Tensor      # [N_grouped]: grouped row -> received row
+    recv_flat_to_row: torch.Tensor      # [N_recv, 1]
+    status: torch.Tensor
+
+
+def dispatch_send(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, ep_size: int,
+                  status: torch.Tensor):
+    """Send side: (send rows [A, H] in destination-rank order, layout,
+    row_to_flat, flat_to_row, count matrix [ep_size, E_local])."""
+    T, K = topk_idx.shape
+    lay = api.dispatch_layout(topk_idx, num_experts, 1, 1, status=status)
+    send, r2f, f2r = api.permute(x, topk_idx, lay, capacity=T * K, status=status)
+    return send, lay, r2f, f2r, count_matrix(lay.tokens_per_expert, ep_size)
+
+
+def dispatch_recv(recv_rows: torch.Tensor, plan: SplitPlan, align: int, status: torch.Tensor):
+    """Receive side: (expert-grouped rows [N_recv + E_local*(align-1), H],
+    layout, row_to_flat, flat_to_row) from the rows as they arrived."""
+    n_recv = recv_rows.shape[0]
+    E_local = plan.received_counts.shape[1]
+    labels = api.segment_labels(plan.received_counts.reshape(-1), E_local, n_recv, status=status)
+    rtopk = labels.view(n_recv, 1)
+    rlay = api.dispatch_layout(rtopk, E_local, 1, align, status=status)
+    grouped, rr2f, rf2r = api.permute(recv_rows, rtopk, rlay, status=status)
+    return grouped, rlay, rr2f, rf2r
+
+
+def combine_send(y_grouped: torch.Tensor, handle: EPHandle) -> torch.Tensor:
+    """Expert outputs back into received order (a unit-weight top_k = 1
+    combine: an exact copy of each row)."""
+    return api.combine_weighted(y_grouped, handle.recv_flat_to_row, None, status=handle.status)
+
+
+def combine_recv(back_rows: torch.Tensor, handle: EPHandle, weights: torch.Tensor,
+                 validate: bool = False) -> torch.Tensor:
+    """fused_weighted_restore of the rows returned in send order."""
+    return api.combine_weighted(back_rows, handle.send_flat_to_row, weights,
+                                row_to_flat=handle.send_row_to_flat, validate=validate,
+                                status=handle.status)
+
+
+def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, align: int = 1,
+                group=None, status: torch.Tensor | None = None):
+    """Dispatch across the ranks of `group` (one GPU each): returns this
+    rank's expert-grouped rows for its local experts and the handle.  Two
+    all-to-alls (counts, rows) and one device-to-host copy (the splits)."""
+    ep_size = dist.get_world_size(group)
+    st = status if status is not None else api.new_status(x.device)
+    send, lay, r2f, f2r, cm = dispatch_send(x, topk_idx, num_experts, ep_size, st)
+    plan = split_plan(cm, group)
+    recv = torch.empty(sum(plan.output_splits), x.shape[1], dtype=x.dtype, device=x.device)
+    dist.all_to_all_single(recv, send[:sum(plan.input_splits)], plan.output_splits,
+                           plan.input_splits, group=group)
+    grouped, rlay, rr2f, rf2r = dispatch_recv(recv, plan, align, st)
+    return grouped, EPHandle(lay, r2f, f2r, plan, rlay, rr2f, rf2r, st)
+
+
+def ep_combine(y_grouped: torch.Tensor, handle: EPHandle, weights: torch.Tensor, group=None,
+               validate: bool = False) -> torch.Tensor:
+    """Combine across the ranks of `group`: the expert outputs go back to
+    their source ranks (one all-to-all) and are restored there."""
+    back = combine_send(y_grouped, handle)
+    plan = handle.plan
+    A = handle.send_row_to_flat.shape[0]
+    returned = torch.empty(A, y_grouped.shape[1], dtype=y_grouped.dtype, device=y_grouped.device)
+    dist.all_to_all_single(returned[:sum(plan.input_splits)], back, plan.input_splits,
+                           plan.output_splits, group=group)
+    return combine_recv(returned, handle, weights, validate)

@@ -320,6 +320,29 @@ int moe_combine_backward_f32(const float* grad_out, const float* rows, int64_t N
 int moe_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
                            int32_t* flat_to_row, int32_t* status, cudaStream_t stream);
 
+/* Row labels from segment counts: the receive side of expert parallelism
+ * across GPUs ([DS-8190] Redundancy: received_counts[s, e] is the number of
+ * rows source rank s sends to local expert e; after the payload all-to-all
+ * they arrive source by source, each source's rows in local-expert order).
+ * Row i of a buffer of n consecutive segments, segment j holding counts[j]
+ * rows, gets
+ *
+ *   labels[i] = j % modulo        (received buffer: j = s*E_local + e,
+ *                                  modulo = E_local, label = local expert)
+ *
+ * and rows past sum(counts) get -1.  The labels, read as topk_idx [rows, 1],
+ * let moe_dispatch_layout + moe_permute regroup the received rows by local
+ * expert (stable: source rank, then the source's order).
+ * In:  counts [n] int32 (device), 1 <= n <= MOE_MAX_E, modulo >= 1,
+ *      0 <= rows <= INT32_MAX.
+ * Out: labels [rows] int64 (device, 8-byte aligned).
+ * Status: MOE_ST_CAPACITY if sum(counts) > rows (the rows past `rows` are not
+ *         labelled), MOE_ST_COVERAGE if a count is negative (counted as 0).
+ * Errors: MOE_ERR_INVALID_ARG for sizes outside the limits, a null pointer or
+ *         misalignment.  One kernel. */
+int moe_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows, int64_t* labels,
+                       int32_t* status, cudaStream_t stream);
+
 /* Backward of fused_weighted_restore ([DS-8847] Tests: row and score
  * gradients; Benchmark: score gradient in FP32; [DeepEP-272]: the backward
  * of combine is a dispatch).  With g = grad_out [T,H]:

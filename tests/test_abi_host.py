@@ -129,6 +129,17 @@ def test_combine_backward_host_checks(L, kw):
     assert rc == -1
 
 
+@pytest.mark.parametrize("kw", [dict(n=0), dict(n=1025), dict(modulo=0), dict(rows=-1),
+                                dict(counts=0), dict(labels=0), dict(labels=A16 + 4),
+                                dict(counts=A16 + 2), dict(status=0)])
+def test_segment_labels_host_checks(L, kw):
+    a = dict(counts=A16, n=32, modulo=8, rows=100, labels=A16, status=A16)
+    a.update(kw)
+    rc = L.moe_segment_labels(a["counts"], a["n"], a["modulo"], a["rows"], a["labels"],
+                              a["status"], None)
+    assert rc == -1
+
+
 def test_expert_scale_host_checks(L):
     assert L.moe_expert_scale(A16, 256, A16, A16, 8, 64, A16, A16, A16, None) == -1  # aliasing
     assert L.moe_expert_scale(A16, 256, A16, A16, 0, 64, A16, A16 + 16, A16, None) == -1

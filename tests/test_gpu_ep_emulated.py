@@ -1,0 +1,98 @@
+"""Dispatch and combine across R ranks, emulated in one process on one GPU.
+
+Every rank's send and receive steps run in the library's kernels (layout,
+permute, segment labels, combine); the exchanges between ranks are plain
+tensor copies of exactly what all_to_all_single would deliver, so no kernel
+waits on another.  Against the single-device path with the ranks as logical
+groups: every rank's plan equals the single-device count matrix and splits,
+the expert-grouped rows of every local expert are bit-identical to that
+expert's rows there (pads zero), and the combined output of every rank's
+tokens is bit-identical to the single-device output."""
+import numpy as np
+import pytest
+import torch
+
+from combine_moe_dispatch_03_b200.inputs import custom_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from combine_moe_dispatch_03_b200 import build
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _i16(t):
+    return t.contiguous().view(torch.int16)
+
+
+@pytest.mark.parametrize("R,E,K,Tb,H,align,skew", [
+    (4, 32, 4, 512, 256, 8, 0.0),
+    (8, 64, 8, 256, 136, 16, 3.0),      # ragged rows (17 vectors), severe skew
+    (2, 8, 2, 300, 64, 1, 0.0),         # no padding
+])
+def test_ep_dispatch_combine_emulated(R, E, K, Tb, H, align, skew):
+    from combine_moe_dispatch_03_b200 import api, ep
+    dev = torch.device("cuda:0")
+    T, El = R * Tb, E // R
+    g = torch.Generator().manual_seed(R * 1000 + E + K)
+    logits = torch.randn(T, E, generator=g)
+    if skew:
+        rank = torch.randperm(E, generator=g).double() + 1.0
+        logits += (skew * torch.log(rank ** -1.2 / (rank ** -1.2).sum())).float()
+    topk = torch.topk(logits, K, dim=1).indices
+    inp = custom_inputs(T, H, E, K, seed=R + E, topk_idx=topk)
+    x, w, tk = inp["x"].to(dev), inp["weights"].to(dev), topk.to(dev)
+    st = api.new_status(dev)
+
+    # single device, ranks as logical groups
+    lay = api.dispatch_layout(tk, E, R, align, status=st)
+    xp, _, f2r = api.permute(x, tk, lay, status=st)
+    out_ref = api.combine_weighted(xp * 2, f2r, w, status=st)
+    off = lay.expert_offsets.cpu().tolist()
+    cnt = lay.tokens_per_expert.cpu().tolist()
+    counts_all = lay.counts.cpu()
+    splits_all = lay.splits.cpu()
+
+    # send side of every rank
+    sends = [ep.dispatch_send(x[r * Tb:(r + 1) * Tb].contiguous(),
+                              tk[r * Tb:(r + 1) * Tb].contiguous(), E, R, st) for r in range(R)]
+    # count exchange: rank r receives row r of every rank's count matrix
+    plans = []
+    for r in range(R):
+        received = torch.stack([sends[s][4][r] for s in range(R)]).to(torch.int32).contiguous()
+        plans.append(ep.plan_from_counts(sends[r][4].to(torch.int32), received))
+        assert torch.equal(plans[r].received_counts.cpu(), counts_all[:, r, :])
+        assert plans[r].input_splits == splits_all[r, :].tolist()
+        assert plans[r].output_splits == splits_all[:, r].tolist()
+    # row exchange: rank r receives, source by source, the rows each sends to r
+    starts = [np.concatenate([[0], np.cumsum(p.input_splits)]) for p in plans]
+    handles, grouped = [], []
+    for r in range(R):
+        parts = [sends[s][0][starts[s][r]:starts[s][r + 1]] for s in range(R)]
+        recv = torch.cat(parts).contiguous()
+        assert recv.shape[0] == sum(plans[r].output_splits)
+        gr, rlay, rr2f, rf2r = ep.dispatch_recv(recv, plans[r], align, st)
+        handles.append(ep.EPHandle(sends[r][1], sends[r][2], sends[r][3], plans[r], rlay, rr2f,
+                                   rf2r, st))
+        grouped.append(gr)
+        roff = rlay.expert_offsets.cpu().tolist()
+        for el in range(El):
+            e, c = r * El + el, cnt[r * El + el]
+            assert roff[el + 1] - roff[el] == off[e + 1] - off[e]
+            assert torch.equal(_i16(gr[roff[el]:roff[el] + c]), _i16(xp[off[e]:off[e] + c])), e
+            assert not _i16(gr[roff[el] + c:roff[el + 1]]).any()
+    # experts, then the reverse exchange and the restore on every source rank
+    backs = [ep.combine_send(grouped[r] * 2, handles[r]) for r in range(R)]
+    rstarts = [np.concatenate([[0], np.cumsum(p.output_splits)]) for p in plans]
+    for s in range(R):
+        returned = torch.empty(Tb * K, H, dtype=torch.bfloat16, device=dev)
+        parts = torch.cat([backs[r][rstarts[r][s]:rstarts[r][s + 1]] for r in range(R)])
+        returned[:parts.shape[0]] = parts
+        out_s = ep.combine_recv(returned, handles[s], w[s * Tb:(s + 1) * Tb].contiguous(),
+                                validate=True)
+        assert torch.equal(_i16(out_s), _i16(out_ref[s * Tb:(s + 1) * Tb])), s
+    api.check_status(st)

@@ -56,3 +56,30 @@ def test_split_plan_from_expert_indices_nccl_one_rank():
         assert plan.received_counts.sum(dim=1).tolist() == plan.output_splits
     finally:
         dist.destroy_process_group()
+
+
+def test_ep_dispatch_combine_nccl_one_rank():
+    """ep_dispatch / ep_combine through NCCL with one rank: equal, bit for
+    bit, to the single-device layout, permute and restore."""
+    import torch.distributed as dist
+    from combine_moe_dispatch_03_b200 import api, ep
+    cfg = CONFIGS["qwen3"]
+    inp = make_inputs("qwen3", T=2048)
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        x, tk, w = inp["x"].to(dev), inp["topk_idx"].to(dev), inp["weights"].to(dev)
+        st = api.new_status(dev)
+        lay = api.dispatch_layout(tk, cfg.E, 1, cfg.align, status=st)
+        xp, _, f2r = api.permute(x, tk, lay, status=st)
+        out_ref = api.combine_weighted(xp * 2, f2r, w, status=st)
+        grouped, h = ep.ep_dispatch(x, tk, cfg.E, cfg.align, status=st)
+        n_pad = int(lay.expert_offsets[-1])
+        assert torch.equal(grouped[:n_pad].view(torch.int16), xp[:n_pad].view(torch.int16))
+        out = ep.ep_combine(grouped * 2, h, w, validate=True)
+        assert torch.equal(out.view(torch.int16), out_ref.view(torch.int16))
+        api.check_status(st)
+    finally:
+        dist.destroy_process_group()

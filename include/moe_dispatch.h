@@ -11,6 +11,12 @@
  *   moe_combine_backward  row gradients + routing-weight grads   (fp32 / fp64)
  *   moe_combine_weighted  with weights = NULL: dispatch backward (fp32 accumulate)
  *
+ * Variants and helpers: moe_dispatch_layout_noalloc (no workspace argument),
+ * moe_permute_payload (FP8 (data, scales) or any row payload),
+ * moe_combine_weighted_f32 / moe_combine_backward_f32 (fp32 rows),
+ * moe_scatter_flat_index (the folded restore's scatter), moe_segment_labels
+ * (the receive side of expert parallelism across ranks).
+ *
  * Sources (titles of the pages that define the operations):
  *   [DeepEP-272] DeepEP issue "Does Deepep's Dispatch/Combine Support Autograd
  *                Like PyTorch's all_to_all?": get_dispatch_layout and its

@@ -360,7 +360,10 @@ def run_ours(args, cfg, inp, dist, rank, ws, device):
                      "traffic": ncu_traffic(dom, cfg.name), "bytes_per_launch": dom_bytes,
                      "mean_ms": dom_mean_ms, "peak_kind": peak_kind},
         "kernels": {n: {"mean_ms": mean_k[n], "share": share[n],
-                        "gbs": nbytes[n] / (mean_k[n] / 1e3) / 1e9} for n in Path.names},
+                        "gbs": nbytes[n] / (mean_k[n] / 1e3) / 1e9,
+                        "frac": nbytes[n] / (mean_k[n] / 1e3) / 1e9 / peak,
+                        "bytes_per_launch": nbytes[n],
+                        "traffic": ncu_traffic(n, cfg.name)} for n in Path.names},
         "eager": eager,
         "e2e": e2e,
         "gpu_launches": Path.kernels_per_step * args.steps,

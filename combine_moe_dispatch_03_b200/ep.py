@@ -1,4 +1,5 @@
-"""Split plan for expert parallelism across processes (one GPU per rank).
+"""Expert parallelism across processes (one GPU per rank): the split plan,
+then dispatch and combine around the row exchange.
 
 Source: DeepSpeed PR "Derive AutoEP rank splits from the per-expert count
 exchange" (Redundancy, Fix, Tests).  Each rank knows how many of its own
@@ -12,11 +13,11 @@ computed from the other.  The two split vectors come to the host in ONE
 device-to-host copy (the payload all-to-all needs them as host integers).
 
 On one GPU the library's layout computes the same quantities for all logical
-ranks at once (counts [R, R, E_local], splits [R, R]); this module is the
-exchange step a real multi-GPU deployment puts between the layout and the
-payload all-to-all.  It is host plumbing over torch.distributed (NCCL on
-GPUs, gloo on CPU); the per-expert counts of split_plan_from_expert_indices
-come from the library's layout kernel.
+ranks at once (counts [R, R, E_local], splits [R, R]); this module is what a
+multi-GPU deployment puts around the exchanges: the split plan, then the
+rows (see the section "the payload across ranks" below).  Every step on the
+rows runs in the library's kernels; the exchanges are torch.distributed
+all-to-alls (NCCL on GPUs; the split plan also runs over gloo on CPU).
 """
 from __future__ import annotations
 

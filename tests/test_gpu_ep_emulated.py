@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from combine_moe_dispatch_03_b200.inputs import custom_inputs
+from combine_moe_dispatch_03_b200.inputs import CONFIGS, custom_inputs, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -35,17 +35,31 @@ def _i16(t):
     (2, 8, 2, 300, 64, 1, 0.0),         # no padding
 ])
 def test_ep_dispatch_combine_emulated(R, E, K, Tb, H, align, skew):
-    from combine_moe_dispatch_03_b200 import api, ep
-    dev = torch.device("cuda:0")
-    T, El = R * Tb, E // R
+    T = R * Tb
     g = torch.Generator().manual_seed(R * 1000 + E + K)
     logits = torch.randn(T, E, generator=g)
     if skew:
         rank = torch.randperm(E, generator=g).double() + 1.0
         logits += (skew * torch.log(rank ** -1.2 / (rank ** -1.2).sum())).float()
     topk = torch.topk(logits, K, dim=1).indices
-    inp = custom_inputs(T, H, E, K, seed=R + E, topk_idx=topk)
-    x, w, tk = inp["x"].to(dev), inp["weights"].to(dev), topk.to(dev)
+    _run_emulated(custom_inputs(T, H, E, K, seed=R + E, topk_idx=topk), R, E, align)
+
+
+@pytest.mark.parametrize("name", ["dsv3", "dsv3_skew"])
+def test_ep_dispatch_combine_emulated_full_size(name):
+    """The DeepSeek-V3-shaped workloads at full size (8 ranks x 1024 tokens,
+    256 experts, top-8, H 7168, align 128), their seeded routing."""
+    cfg = CONFIGS[name]
+    _run_emulated(make_inputs(name), cfg.R, cfg.E, cfg.align)
+
+
+def _run_emulated(inp, R, E, align):
+    from combine_moe_dispatch_03_b200 import api, ep
+    dev = torch.device("cuda:0")
+    T, K = inp["topk_idx"].shape
+    H = inp["x"].shape[1]
+    Tb, El = T // R, E // R
+    x, w, tk = inp["x"].to(dev), inp["weights"].to(dev), inp["topk_idx"].to(dev)
     st = api.new_status(dev)
 
     # single device, ranks as logical groups

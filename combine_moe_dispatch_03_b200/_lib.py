@@ -54,6 +54,9 @@ SIGNATURES = {
                                       _P, _P]),
     "moe_scatter_flat_index": (_I, [_P, _L, _I, _I, _P, _P, _P]),
     "moe_segment_labels": (_I, [_P, _I, _I, _L, _P, _P, _P]),
+    "moe_permute_to_ranks": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _L, _I, _P, _P, _I, _P,
+                                  _P, _P]),
+    "moe_combine_from_ranks": (_I, [_P, _I, _L, _P, _P, _I, _P, _I, _I, _I, _I, _P, _P, _P]),
     "moe_strerror": (ctypes.c_char_p, [_I]),
     "moe_status_bit_name": (ctypes.c_char_p, [_I]),
     "moe_version": (ctypes.c_char_p, []),

@@ -270,6 +270,47 @@ int moe_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows, i
     return finish(moe::launch_segment_labels(counts, n, modulo, rows, labels, status, stream));
 }
 
+int moe_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int R,
+                         int H, const int32_t* dest_base, const void* workspace,
+                         uint16_t* const* dest_rows, int64_t dest_cap, int rank,
+                         const int32_t* own_offsets, const int32_t* own_counts, int zero_pad,
+                         int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
+    NvtxRange range("moe_permute_to_ranks");
+    if (!sizes_ok(T, K, E) || !hidden_ok(H) || R < 1 || R > MOE_MAX_R || E % R || rank < 0 ||
+        rank >= R || dest_cap < 0 || dest_cap > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (!dest_base || !workspace || !dest_rows || !own_offsets || !own_counts || !status)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !topk_idx || !flat_to_row)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(topk_idx, 8) || !aligned(workspace, 16) ||
+        !aligned(dest_rows, 8) || !aligned(dest_base, 4) || !aligned(own_offsets, 4) ||
+        !aligned(own_counts, 4) || !aligned(flat_to_row, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    return finish(moe::launch_permute_to_ranks(x, topk_idx, T, K, E, R, H, dest_base, workspace,
+                                               dest_rows, dest_cap, rank, own_offsets, own_counts,
+                                               zero_pad, flat_to_row, status, stream));
+}
+
+int moe_combine_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
+                           const int32_t* flat_to_row, const int64_t* topk_idx, int E,
+                           const void* weights, int weight_dtype, int T, int K, int H,
+                           uint16_t* out, int32_t* status, cudaStream_t stream) {
+    NvtxRange range("moe_combine_from_ranks");
+    if (!sizes_ok(T, K, E) || !hidden_ok(H) || R < 1 || R > MOE_MAX_R || E % R || N_cap < 0 ||
+        N_cap > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (weight_dtype != MOE_DTYPE_F32 && weight_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (!status || !rows) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!flat_to_row || !topk_idx || !weights || !out)) return MOE_ERR_INVALID_ARG;
+    const size_t wal = weight_dtype == MOE_DTYPE_F32 ? 4 : 2;
+    if (!aligned(rows, 8) || !aligned(flat_to_row, 4) || !aligned(topk_idx, 8) ||
+        !aligned(weights, wal) || !aligned(out, 16) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    return finish(moe::launch_combine_from_ranks(rows, R, N_cap, flat_to_row, topk_idx, E, weights,
+                                                 weight_dtype, T, K, H, out, status, stream));
+}
+
 const char* moe_strerror(int code) {
     switch (code) {
         case MOE_OK: return "ok";

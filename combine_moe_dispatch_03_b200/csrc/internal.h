@@ -129,6 +129,18 @@ cudaError_t launch_combine_backward_f32(const float* grad_out, const float* rows
 cudaError_t launch_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
                                       int32_t* flat_to_row, int32_t* status, cudaStream_t stream);
 
+cudaError_t launch_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int K,
+                                    int E, int R, int H, const int32_t* dest_base,
+                                    const void* workspace, uint16_t* const* dest_rows,
+                                    int64_t dest_cap, int rank, const int32_t* own_offsets,
+                                    const int32_t* own_counts, int zero_pad, int32_t* flat_to_row,
+                                    int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_combine_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
+                                      const int32_t* flat_to_row, const int64_t* topk_idx, int E,
+                                      const void* weights, int weight_dtype, int T, int K, int H,
+                                      uint16_t* out, int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows,
                                   int64_t* labels, int32_t* status, cudaStream_t stream);
 

@@ -175,3 +175,81 @@ def ep_combine(y_grouped: torch.Tensor, handle: EPHandle, weights: torch.Tensor,
     dist.all_to_all_single(returned[:sum(plan.input_splits)], back, plan.input_splits,
                            plan.output_splits, group=group)
     return combine_recv(returned, handle, weights, validate)
+
+
+# ------------------------------------- the payload without a send buffer ---
+#
+# The fused form: every rank stores its rows straight into the receive
+# buffers of the ranks that own their experts (moe_permute_to_ranks), and
+# gathers the expert outputs straight from them (moe_combine_from_ranks).
+# The buffers are reached through a table of addresses, one per rank --
+# across GPUs, the peer addresses of buffers every rank has mapped (e.g. with
+# CUDA IPC or symmetric memory; the mapping itself is the caller's).  Only
+# the per-expert counts are exchanged (an all-gather of [E] per rank); the
+# rows cross the interconnect once, inside the kernels.  The caller puts a
+# barrier between the dispatch and the experts' reads of the buffers, and
+# between the experts' writes and the combine.
+
+
+def rank_bases(all_counts: torch.Tensor, rank: int, align: int = 1):
+    """From the per-expert counts of every source rank ([ep_size, E], row s =
+    rank s's tokens_per_expert): (dest_base [E] -- the row where `rank`'s
+    rows of expert e start in e's owner's buffer --, own_offsets
+    [E_local + 1] -- the padded group starts in `rank`'s own buffer --,
+    own_counts [E_local] -- the real rows of each of its groups).  Metadata
+    arithmetic on [ep_size, E] integers."""
+    R, E = all_counts.shape
+    El = E // R
+    c = all_counts.to(torch.int64)
+    total = c.sum(dim=0)                                          # rows of e from all ranks
+    padded = ((total + align - 1) // align * align).view(R, El)
+    start = torch.cumsum(padded, dim=1) - padded                  # group starts per owner
+    before = c[:rank].sum(dim=0)                                  # rows of e from earlier ranks
+    dest_base = (start.reshape(E) + before).to(torch.int32)
+    own_offsets = torch.cat([start[rank], padded[rank].sum().view(1)]).to(torch.int32)
+    own_counts = total.view(R, El)[rank].to(torch.int32)
+    return dest_base.contiguous(), own_offsets.contiguous(), own_counts.contiguous()
+
+
+def direct_receive_rows(all_counts: torch.Tensor, align: int = 1) -> int:
+    """Rows every rank's receive buffer needs for this routing (the largest
+    padded total over the ranks).  One device-to-host copy."""
+    R, E = all_counts.shape
+    total = all_counts.to(torch.int64).sum(dim=0)
+    padded = ((total + align - 1) // align * align).view(R, E // R)
+    return int(padded.sum(dim=1).max().item())
+
+
+@dataclasses.dataclass
+class DirectHandle:
+    layout: api.Layout            # this rank's tokens, one source block
+    flat_to_row: torch.Tensor     # [T, K]: row in the buffer of each slot's expert rank
+    own_offsets: torch.Tensor     # [E_local + 1]: this rank's groups in its own buffer
+    own_counts: torch.Tensor      # [E_local]
+    status: torch.Tensor
+
+
+def ep_dispatch_direct(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int,
+                       dest_table: torch.Tensor, dest_cap: int, align: int = 1, group=None,
+                       status: torch.Tensor | None = None) -> DirectHandle:
+    """Dispatch into the receive buffers listed in dest_table (one address
+    per rank of `group`, each buffer [dest_cap, H] bf16).  One all-gather of
+    the per-expert counts; the rows go out inside the permute."""
+    R, rank = dist.get_world_size(group), dist.get_rank(group)
+    st = status if status is not None else api.new_status(x.device)
+    lay = api.dispatch_layout(topk_idx, num_experts, 1, 1, status=st)
+    all_counts = torch.empty(R, num_experts, dtype=torch.int32, device=x.device)
+    dist.all_gather_into_tensor(all_counts, lay.tokens_per_expert, group=group)
+    dest_base, own_off, own_cnt = rank_bases(all_counts, rank, align)
+    f2r = api.permute_to_ranks(x, topk_idx, lay, dest_base, dest_table, dest_cap, rank, own_off,
+                               own_cnt, status=st)
+    return DirectHandle(lay, f2r, own_off, own_cnt, st)
+
+
+def ep_combine_direct(rows_table: torch.Tensor, N_cap: int, H: int, handle: DirectHandle,
+                      topk_idx: torch.Tensor, weights: torch.Tensor) -> torch.Tensor:
+    """fused_weighted_restore of this rank's tokens, each slot read from the
+    expert-output buffer of its expert's rank (rows_table: one address per
+    rank)."""
+    return api.combine_from_ranks(rows_table, N_cap, H, handle.flat_to_row, topk_idx,
+                                  handle.layout.E, weights, status=handle.status)

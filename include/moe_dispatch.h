@@ -15,7 +15,9 @@
  * moe_permute_payload (FP8 (data, scales) or any row payload),
  * moe_combine_weighted_f32 / moe_combine_backward_f32 (fp32 rows),
  * moe_scatter_flat_index (the folded restore's scatter), moe_segment_labels
- * (the receive side of expert parallelism across ranks).
+ * (the receive side of expert parallelism across ranks), moe_permute_to_ranks
+ * and moe_combine_from_ranks (dispatch into / combine out of the ranks'
+ * buffers directly, through peer pointers).
  *
  * Sources (titles of the pages that define the operations):
  *   [DeepEP-272] DeepEP issue "Does Deepep's Dispatch/Combine Support Autograd
@@ -348,6 +350,63 @@ int moe_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
  *         misalignment.  One kernel. */
 int moe_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows, int64_t* labels,
                        int32_t* status, cudaStream_t stream);
+
+/* Dispatch straight into the receive buffers of the ranks that own the
+ * experts (expert parallelism across GPUs without a send buffer; [DeepEP-272]
+ * dispatch sends token rows to the ranks owning their experts; [DS-8190] the
+ * per-(source rank, expert) counts the offsets come from).  Rank `rank` of R,
+ * holding T tokens, stores assignment f = (t, k) of expert e into the buffer
+ * of rank r = e / (E/R) at
+ *
+ *   row(f) = dest_base[e] + #{f' < f of this rank's tokens : topk_idx[f'] = e}
+ *
+ * where dest_base[e] = (start of e's padded group in rank r's buffer) + (rows
+ * of e sent by ranks before `rank`), so every receive buffer comes out in the
+ * order the single-device layout gives those experts (source rank, token,
+ * slot), padded per expert to the group alignment.  The pad rows of this
+ * rank's OWN receive buffer are zeroed here when zero_pad != 0 (every rank
+ * zeroes its own).
+ * In:  x [T,H] bf16, topk_idx [T,K] int64, dest_base [E] int32 (device),
+ *      workspace: moe_dispatch_layout of these T tokens with R = 1 (its
+ *      in-tile ranks; checked on the device: MOE_ST_LAYOUT_MISMATCH),
+ *      dest_rows: DEVICE array of R pointers to bf16 buffers [dest_cap, H]
+ *      (16-byte aligned; across GPUs, peer addresses of the other ranks'
+ *      buffers, written with plain stores), own_offsets [E/R + 1] and
+ *      own_counts [E/R] int32: this rank's padded group starts and real rows.
+ * Out: the rows in the ranks' buffers; flat_to_row [T,K] int32 = row(f) in
+ *      the buffer of its expert's rank (-1 if none).
+ * Status: MOE_ST_EXPERT_OOR, MOE_ST_CAPACITY (a row at or past dest_cap is
+ *         not written), MOE_ST_LAYOUT_MISMATCH.
+ * Errors: MOE_ERR_INVALID_ARG for sizes outside the limits (also E % R,
+ *         rank outside [0, R)), a null pointer or misalignment.  The caller
+ *         orders the ranks' calls before any reader of the buffers (across
+ *         GPUs: a barrier between this call and the experts). */
+int moe_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int R,
+                         int H, const int32_t* dest_base, const void* workspace,
+                         uint16_t* const* dest_rows, int64_t dest_cap, int rank,
+                         const int32_t* own_offsets, const int32_t* own_counts, int zero_pad,
+                         int32_t* flat_to_row, int32_t* status, cudaStream_t stream);
+
+/* Combine straight out of the ranks' expert-output buffers: the
+ * fused_weighted_restore of [DS-8847] for this rank's T tokens, slot (t, k)
+ * read from the buffer of rank topk_idx[t,k] / (E/R) at row flat_to_row[t,k]
+ * (as moe_permute_to_ranks wrote it):
+ *
+ *   out[t] = bf16_rn(fmaf chain over k of w[t,k] * rows[rank][flat_to_row[t,k]])
+ *
+ * the same FP32 slot-order chain as moe_combine_weighted, so the result is
+ * bit-identical to the single-device restore of the same rows.
+ * In:  rows: DEVICE array of R pointers to bf16 [N_cap, H] buffers (across
+ *      GPUs, peer addresses; plain loads), flat_to_row [T,K], topk_idx [T,K],
+ *      weights [T,K] fp32 or bf16.
+ * Out: out [T,H] bf16.
+ * Status: MOE_ST_ROW_OOR for a slot whose row or expert is out of range (it
+ *         contributes nothing).
+ * Errors: MOE_ERR_INVALID_ARG as moe_combine_weighted, plus E % R. */
+int moe_combine_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
+                           const int32_t* flat_to_row, const int64_t* topk_idx, int E,
+                           const void* weights, int weight_dtype, int T, int K, int H,
+                           uint16_t* out, int32_t* status, cudaStream_t stream);
 
 /* Backward of fused_weighted_restore ([DS-8847] Tests: row and score
  * gradients; Benchmark: score gradient in FP32; [DeepEP-272]: the backward

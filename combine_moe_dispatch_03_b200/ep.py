@@ -220,6 +220,19 @@ def direct_receive_rows(all_counts: torch.Tensor, align: int = 1) -> int:
     return int(padded.sum(dim=1).max().item())
 
 
+def direct_plan(tokens_per_expert: torch.Tensor, group=None, align: int = 1):
+    """The metadata of the direct dispatch: ONE all-gather of every rank's
+    per-expert counts [E], then rank_bases for this rank.  Returns
+    (all_counts [ep_size, E], dest_base, own_offsets, own_counts)."""
+    R, rank = dist.get_world_size(group), dist.get_rank(group)
+    E = tokens_per_expert.numel()
+    all_counts = torch.empty(R, E, dtype=torch.int32, device=tokens_per_expert.device)
+    dist.all_gather_into_tensor(all_counts.view(-1),
+                                tokens_per_expert.to(torch.int32).contiguous().view(-1),
+                                group=group)
+    return (all_counts,) + rank_bases(all_counts, rank, align)
+
+
 @dataclasses.dataclass
 class DirectHandle:
     layout: api.Layout            # this rank's tokens, one source block
@@ -235,12 +248,10 @@ def ep_dispatch_direct(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int
     """Dispatch into the receive buffers listed in dest_table (one address
     per rank of `group`, each buffer [dest_cap, H] bf16).  One all-gather of
     the per-expert counts; the rows go out inside the permute."""
-    R, rank = dist.get_world_size(group), dist.get_rank(group)
+    rank = dist.get_rank(group)
     st = status if status is not None else api.new_status(x.device)
     lay = api.dispatch_layout(topk_idx, num_experts, 1, 1, status=st)
-    all_counts = torch.empty(R, num_experts, dtype=torch.int32, device=x.device)
-    dist.all_gather_into_tensor(all_counts, lay.tokens_per_expert, group=group)
-    dest_base, own_off, own_cnt = rank_bases(all_counts, rank, align)
+    _, dest_base, own_off, own_cnt = direct_plan(lay.tokens_per_expert, group, align)
     f2r = api.permute_to_ranks(x, topk_idx, lay, dest_base, dest_table, dest_cap, rank, own_off,
                                own_cnt, status=st)
     return DirectHandle(lay, f2r, own_off, own_cnt, st)

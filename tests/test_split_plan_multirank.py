@@ -13,9 +13,12 @@ rank splits from the per-expert count exchange":
     [R, R, E_local] and splits [R, R]), and the per-rank totals also match
     an independent direct count.
 
-Each rank's own count matrix comes from the oracle here (no GPU); on a GPU,
-split_plan_from_expert_indices takes it from the library's layout kernel
-(tests/test_gpu_split_plan.py)."""
+The direct (send-buffer-free) dispatch's metadata runs the same way: one
+all-gather of the per-expert counts, then each rank's row bases, checked
+against the oracle's single-device rows.
+
+Each rank's own counts come from the oracle here (no GPU); on a GPU they
+come from the library's layout kernel (tests/test_gpu_split_plan.py)."""
 import datetime
 import os
 import socket
@@ -138,3 +141,60 @@ def test_split_plan_across_processes(ws):
             np.testing.assert_array_equal(o_recv, received)
             np.testing.assert_array_equal(o_pe, per_expert)
             assert (r["n_new"], r["n_old"]) == (1, 2), kind
+
+
+def _direct_worker(rank, ws, port, align, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle as orc
+    from combine_moe_dispatch_03_b200 import ep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        topk = _routing("severe", ws)
+        mine = topk[rank * TB:(rank + 1) * TB]
+        tpe = torch.from_numpy(orc.layout(mine, E, 1, 1)["tokens_per_expert"])
+        all_counts, dest_base, own_off, own_cnt = ep.direct_plan(tpe, align=align)
+        q.put((rank, all_counts.numpy(), dest_base.numpy(), own_off.numpy(), own_cnt.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws,align", [(2, 8), (4, 1)])
+def test_direct_plan_across_processes(ws, align):
+    """The direct dispatch's metadata over real processes: one all-gather of
+    the per-expert counts, then each rank's row bases, which must put every
+    assignment at the oracle's single-device row minus the start of its
+    owner rank's block (the owner's padded groups and real rows likewise)."""
+    import oracle as orc
+    orc.build()
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_direct_worker, args=(r, ws, port, align, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    res = dict((r[0], r[1:]) for r in (q.get(timeout=240) for _ in range(ws)))
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    topk = _routing("severe", ws)
+    El = E // ws
+    lay = orc.layout(topk, E, ws, align)
+    off = lay["expert_offsets"]
+    pm = orc.permute(np.zeros((topk.shape[0], 8), np.uint16), topk, E, off, int(off[-1]))
+    for rank in range(ws):
+        all_counts, dest_base, own_off, own_cnt = res[rank]
+        for s in range(ws):
+            np.testing.assert_array_equal(
+                all_counts[s], orc.layout(topk[s * TB:(s + 1) * TB], E, 1, 1)["tokens_per_expert"])
+        np.testing.assert_array_equal(own_off, off[rank * El:(rank + 1) * El + 1] - off[rank * El])
+        np.testing.assert_array_equal(own_cnt, lay["tokens_per_expert"][rank * El:(rank + 1) * El])
+        seen = np.zeros(E, np.int64)
+        for t in range(rank * TB, (rank + 1) * TB):
+            for k in range(K):
+                e = int(topk[t, k])
+                want = int(pm["flat_to_row"][t, k]) - int(off[(e // El) * El])
+                assert dest_base[e] + seen[e] == want, (rank, t, k)
+                seen[e] += 1

@@ -18,7 +18,9 @@ step captured once in a CUDA graph and replayed per timed step (device time,
 CUDA events around each replay, max over ranks, L2 flushed by a 256 MiB write
 between steps); ``eager`` = the same steps launched one by one with a CUDA
 event between every two kernels, which also gives the per-kernel breakdown
-(``kernels``) and the roofline figure; ``e2e`` = the same through pinned host buffers with the host<->device
+(``kernels``: per kernel its mean time, share of the step, algorithmic GB/s,
+fraction of the measured peak and, while its source is unchanged, the DRAM
+traffic per launch from the committed ncu summary) and the roofline figure; ``e2e`` = the same through pinned host buffers with the host<->device
 copies inside the timed region, ``roofline`` = the dominant kernel's
 algorithmic bytes per launch / its mean event-timed duration against the
 measured HBM copy bandwidth, ``cpu_baseline`` = the CPU oracle on a bounded

@@ -43,3 +43,39 @@ def test_rank_bases_match_single_device_rows(R, E, K, Tb, align, seed):
                 want = int(pm["flat_to_row"][t, k]) - int(off[r * El])
                 assert dest_base[e] + seen[e] == want, (s, t, k)
                 seen[e] += 1
+
+
+def test_rank_bases_tile_every_group_exactly():
+    """Random count matrices (hypothesis): for every expert e, the ranks'
+    row ranges [dest_base_s[e], dest_base_s[e] + counts[s][e]) tile the real
+    rows of e's group in its owner's buffer exactly, in rank order; the
+    groups are aligned, contiguous, padded by less than the alignment and
+    do not overlap; the buffer size is the largest owner's padded total."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=200, deadline=None)
+    @given(R=st.integers(1, 6), El=st.integers(1, 5), align=st.integers(1, 9),
+           data=st.data())
+    def check(R, El, align, data):
+        E = R * El
+        c = np.array(data.draw(st.lists(st.integers(0, 40), min_size=R * E, max_size=R * E)),
+                     np.int32).reshape(R, E)
+        all_counts = torch.from_numpy(c)
+        total = c.sum(axis=0)
+        cap = ep.direct_receive_rows(all_counts, align)
+        owner_sizes = []
+        for s in range(R):
+            base, own_off, own_cnt = (t.numpy() for t in ep.rank_bases(all_counts, s, align))
+            assert own_off[0] == 0 and np.all(np.diff(own_off) >= own_cnt)
+            assert np.all(own_off[:-1] % align == 0)
+            assert np.all(np.diff(own_off) - own_cnt < align)
+            np.testing.assert_array_equal(own_cnt, total[s * El:(s + 1) * El])
+            owner_sizes.append(int(own_off[-1]))
+            for e in range(E):
+                r, el = divmod(e, El)
+                _, r_off, _ = ep.rank_bases(all_counts, r, align)
+                assert base[e] == int(r_off[el]) + int(c[:s, e].sum())
+        assert cap == max(owner_sizes)
+
+    check()

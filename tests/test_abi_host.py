@@ -190,3 +190,25 @@ def test_product_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
                 assert "moe_oracle" not in text, f
+
+
+def test_abi_usable_from_plain_c(tmp_path):
+    """A C program compiled against include/moe_dispatch.h and linked to the
+    library makes host-only calls (sizes, strings, argument checks) and
+    gets the documented answers: the boundary is a C ABI, not a Python one."""
+    import shutil
+    from combine_moe_dispatch_03_b200 import build
+    build.build()
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    lib_dir = os.path.dirname(build.LIB_PATH)
+    exe = str(tmp_path / "abi_from_c")
+    src = os.path.join(ROOT, "tests", "c", "abi_from_c.c")
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", cuda_inc, src, "-o", exe, "-L", lib_dir, "-lmoe_dispatch",
+                    "-Wl,-rpath," + lib_dir], check=True, capture_output=True, text=True)
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    assert "C ABI checks passed" in out.stdout

@@ -79,3 +79,44 @@ def test_rank_bases_tile_every_group_exactly():
         assert cap == max(owner_sizes)
 
     check()
+
+
+@pytest.mark.parametrize("R,E,K,Tb,H,align,seed", [(4, 16, 3, 40, 8, 4, 5), (3, 9, 2, 25, 16, 1, 6),
+                                                   (2, 8, 4, 33, 8, 8, 7)])
+def test_receive_buffers_by_definition(R, E, K, Tb, H, align, seed):
+    """Brute force from the definition of expert parallelism: rank r's
+    receive buffer holds, for each of its experts e in order, the rows
+    x[t] of every assignment (t, k) with topk[t, k] == e, source ranks in
+    order, each source's tokens then slots in order, padded with zeros to the
+    alignment.  That buffer is exactly rows [off[r*E_local], off[(r+1)*E_local])
+    of the oracle's single-device grouped buffer, and rank s's align-1
+    permute of its own tokens is its send buffer: destination rank, local
+    expert, token, slot."""
+    orc.build()
+    rng = np.random.default_rng(seed)
+    T, El = R * Tb, E // R
+    topk = rng.integers(0, E, size=(T, K)).astype(np.int64)
+    x = rng.integers(1, 0x7F00, size=(T, H)).astype(np.uint16)       # distinct-ish, nonzero rows
+    lay = orc.layout(topk, E, R, align)
+    off = lay["expert_offsets"]
+    single = orc.permute(x, topk, E, off, int(off[-1]))["x_perm"]
+    for r in range(R):
+        rows = []
+        for e in range(r * El, (r + 1) * El):
+            n = 0
+            for s in range(R):
+                for t in range(s * Tb, (s + 1) * Tb):
+                    for k in range(K):
+                        if topk[t, k] == e:
+                            rows.append(x[t])
+                            n += 1
+            rows.extend([np.zeros(H, np.uint16)] * ((-n) % align))
+        recv = np.array(rows, np.uint16).reshape(-1, H)
+        np.testing.assert_array_equal(recv, single[off[r * El]:off[(r + 1) * El]])
+    for s in range(R):
+        mine = topk[s * Tb:(s + 1) * Tb]
+        lay_s = orc.layout(mine, E, 1, 1)
+        send = orc.permute(x[s * Tb:(s + 1) * Tb], mine, E, lay_s["expert_offsets"], Tb * K)["x_perm"]
+        want = [x[s * Tb + t] for e in range(E) for t in range(Tb) for k in range(K)
+                if mine[t, k] == e]
+        np.testing.assert_array_equal(send, np.array(want, np.uint16).reshape(-1, H))

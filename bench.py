@@ -1,32 +1,56 @@
-"""Benchmark: one step = the whole MoE dispatch/combine path, forward and
-backward, on synthetic seeded inputs resident in HBM.
+"""Benchmark: MoE dispatch + combine on one B200, on seeded synthetic inputs
+resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload qwen3|dsv3|dsv3_skew|mixtral|tiny|page_k4|page_k8|
                                 page_k4_32k|page_k8_32k]
+                    [--workloads dsv3,dsv3_skew,mixtral|none]
 
-Step (seven kernels, all through the C ABI of libmoe_dispatch.so):
-  layout -> permute -> stand-in experts -> weighted combine
-  -> combine backward -> stand-in backward -> unit-weight combine.
+One step = one pass of the path over one batch.  What is timed (``value``) is
+dispatch + combine, the steps of the metric:
+  forward-only workloads:   layout + permute | combine
+  fwd+bwd workloads:        layout + permute | combine + combine backward |
+                            dispatch backward (a unit-weight combine)
+The seeded stand-in expert (y = x * s_e, and its backward) runs between the
+timed segments -- the combine needs its output -- but outside the CUDA
+events: it stands where the grouped expert GEMMs would and is not part of
+dispatch or combine.
+
+Each segment is captured once in its own CUDA graph and replayed every step.
+Before every timed segment L2 is flushed outside the events (a 256 MiB device
+write, then a 256 MiB read of another buffer, so the segment starts with
+neither useful nor dirty lines in L2); CUDA events on the launching stream
+bracket each timed segment; the step time is the sum of its timed segments;
+``value`` = tokens/s over all ranks (every rank's tokens / the slowest rank's
+total time).
 
 Default workload: Qwen3-MoE-shaped fwd+bwd (T=16384 tokens, H=2048, E=128 in
-8 logical ranks, top_k=8, fp32 router weights, mild skew, align 16): the one
-configuration that runs every step of the path, backward included.
+8 logical ranks, top_k=8, fp32 router weights, mild skew, align 16), the one
+configuration that runs every step of the path.  ``workloads`` adds, in the
+same run and the same JSON line, the DeepSeek-V3-shaped (balanced and severe
+skew) and Mixtral-shaped configurations, each with its tokens/s, step GB/s,
+fraction of the measured HBM peak and its dominant kernel's fraction.
 
-Prints ONE JSON line (rank 0).  ``value`` = tokens/s over all ranks with the
-step captured once in a CUDA graph and replayed per timed step (device time,
-CUDA events around each replay, max over ranks, L2 flushed by a 256 MiB write
-between steps); ``eager`` = the same steps launched one by one with a CUDA
-event between every two kernels, which also gives the per-kernel breakdown
-(``kernels``: per kernel its mean time, share of the step, algorithmic GB/s,
-fraction of the measured peak and, while its source is unchanged, the DRAM
-traffic per launch from the committed ncu summary) and the roofline figure; ``e2e`` = the same through pinned host buffers with the host<->device
-copies inside the timed region, ``roofline`` = the dominant kernel's
-algorithmic bytes per launch / its mean event-timed duration against the
-measured HBM copy bandwidth, ``cpu_baseline`` = the CPU oracle on a bounded
-sample of the same workload (rank 0, N=1).  With --impl reference the CPU
-oracle itself is timed as the reference arm.  N>1 runs independent replicas
-(the path has no exchange step on one device): weak scaling.
+Other keys of the JSON line (rank 0 prints ONE line):
+  kernels      per dispatch/combine kernel: mean time of an eager launch
+               (flushed L2 before it, CUDA events around it), share of the
+               timed work, algorithmic bytes and GB/s, fraction of the
+               measured peak, ncu DRAM traffic per launch while the kernel's
+               source is unchanged since the committed capture;
+  roofline     the dominant dispatch/combine kernel (largest share; the
+               stand-in is never a candidate): algorithmic bytes per launch /
+               mean event-timed duration against the measured HBM copy
+               bandwidth;
+  full_step    the whole path including the stand-in (7 launches for fwd+bwd)
+               captured in one graph, one flush per step;
+  e2e          the full step through pinned host buffers with the
+               host<->device copies inside the timed region;
+  cpu_baseline the CPU oracle on a bounded token sample of the same workload,
+               the same dispatch/combine steps: the plain single-threaded
+               build and the OpenMP build on all host cores (rank 0, N=1).
+With --impl reference the OpenMP oracle itself is timed as the reference arm.
+N>1 runs independent replicas (the path has no exchange step on one device):
+weak scaling.
 """
 from __future__ import annotations
 
@@ -41,13 +65,17 @@ import sys
 import tempfile
 import time
 
-import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
 FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
+
+# The dispatch/combine kernels the metric times, and the stand-in expert
+# launches that run between them untimed.
+METHOD = ("layout", "permute", "combine", "combine_backward", "dispatch_backward")
+STAND_IN = ("expert_scale", "expert_scale_bwd")
 
 # Step names -> the kernel function each launches (for K <= 8; larger K uses
 # the generic combine_kernel / combine_bwd_kernel).
@@ -182,7 +210,9 @@ class ClockSampler:
 # ------------------------------------------------------------------- ours ---
 
 class Path:
-    """Preallocated buffers and the eight launches of one step."""
+    """Preallocated buffers and the launches of one step, grouped into the
+    segments the bench times (dispatch / combine) and the stand-in expert
+    launches between them (run, not timed)."""
 
     def __init__(self, inp, cfg, device):
         from combine_moe_dispatch_03_b200 import api
@@ -190,11 +220,11 @@ class Path:
         self.cfg = cfg
         self.dev = device
         T, H, E, K, R = cfg.T, cfg.H, cfg.E, cfg.K, cfg.R
+        self.backward = bool(cfg.backward)
         self.x = inp["x"].to(device)
         self.topk = inp["topk_idx"].to(device)
         self.w = inp["weights"].to(device)
         self.s = inp["scales"].to(device)
-        self.g = inp["grad_out"].to(device)
         self.N = api.worst_case_rows(T, K, E, cfg.align)
         bf = dict(dtype=torch.bfloat16, device=device)
         self.status = api.new_status(device)
@@ -204,36 +234,70 @@ class Path:
         self.f2r = torch.empty(T, K, dtype=torch.int32, device=device)
         self.y = torch.zeros(self.N, H, **bf)
         self.out = torch.empty(T, H, **bf)
-        self.grad_rows = torch.zeros(self.N, H, **bf)
-        self.grad_w = torch.empty(T, K, dtype=torch.float32, device=device)
-        self.grad_xp = torch.zeros(self.N, H, **bf)
-        self.grad_x = torch.empty(T, H, **bf)
+        if self.backward:
+            self.g = inp["grad_out"].to(device)
+            self.grad_rows = torch.zeros(self.N, H, **bf)
+            self.grad_w = torch.empty(T, K, dtype=torch.float32, device=device)
+            self.grad_xp = torch.zeros(self.N, H, **bf)
+            self.grad_x = torch.empty(T, H, **bf)
 
-    names = ["layout", "permute", "expert_scale", "combine", "combine_backward", "expert_scale_bwd",
-             "dispatch_backward"]
-    kernels_per_step = 7   # layout, permute, 2x expert_scale, 2x combine, combine backward
+    def segments(self):
+        """(segment name, launches, timed) in step order."""
+        seg = [("dispatch", ("layout", "permute"), True),
+               ("expert", ("expert_scale",), False)]
+        if self.backward:
+            seg += [("combine", ("combine", "combine_backward"), True),
+                    ("expert_bwd", ("expert_scale_bwd",), False),
+                    ("dispatch_backward", ("dispatch_backward",), True)]
+        else:
+            seg += [("combine", ("combine",), True)]
+        return seg
 
-    def step(self, events=None):
-        api, c = self.api, self.cfg
-        st = self.status
-        ev = (lambda i: events[i].record()) if events is not None else (lambda i: None)
-        ev(0)
-        api.dispatch_layout(self.topk, c.E, c.R, c.align, status=st, out=self.lay)
-        ev(1)
-        api.permute(self.x, self.topk, self.lay, capacity=self.N, status=st,
-                    out=(self.xp, self.r2f, self.f2r))
-        ev(2)
-        api.expert_scale(self.xp, self.lay, self.s, status=st, out=self.y)
-        ev(3)
-        api.combine_weighted(self.y, self.f2r, self.w, status=st, out=self.out)
-        ev(4)
-        api.combine_backward(self.g, self.y, self.r2f, self.f2r, self.w, self.lay, status=st,
-                             out=(self.grad_rows, self.grad_w))
-        ev(5)
-        api.expert_scale(self.grad_rows, self.lay, self.s, status=st, out=self.grad_xp)
-        ev(6)
-        api.combine_weighted(self.grad_xp, self.f2r, None, status=st, out=self.grad_x)
-        ev(7)
+    def launches(self):
+        return [n for _, calls, _ in self.segments() for n in calls]
+
+    def method_launches(self):
+        return [n for n in self.launches() if n in METHOD]
+
+    def call(self, name):
+        api, c, st = self.api, self.cfg, self.status
+        if name == "layout":
+            api.dispatch_layout(self.topk, c.E, c.R, c.align, status=st, out=self.lay)
+        elif name == "permute":
+            api.permute(self.x, self.topk, self.lay, capacity=self.N, status=st,
+                        out=(self.xp, self.r2f, self.f2r))
+        elif name == "expert_scale":
+            api.expert_scale(self.xp, self.lay, self.s, status=st, out=self.y)
+        elif name == "combine":
+            api.combine_weighted(self.y, self.f2r, self.w, status=st, out=self.out)
+        elif name == "combine_backward":
+            api.combine_backward(self.g, self.y, self.r2f, self.f2r, self.w, self.lay, status=st,
+                                 out=(self.grad_rows, self.grad_w))
+        elif name == "expert_scale_bwd":
+            api.expert_scale(self.grad_rows, self.lay, self.s, status=st, out=self.grad_xp)
+        elif name == "dispatch_backward":
+            api.combine_weighted(self.grad_xp, self.f2r, None, status=st, out=self.grad_x)
+        else:
+            raise KeyError(name)
+
+    def step(self):
+        for n in self.launches():
+            self.call(n)
+
+
+class Flush:
+    """Evicts L2 outside the timed events: a 256 MiB write, then a 256 MiB
+    read of a second buffer, so the next timed launch finds neither its own
+    data nor dirty lines (whose write-back it would pay for) in L2."""
+
+    def __init__(self, device):
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self.acc = torch.zeros((), dtype=torch.float32, device=device)
+
+    def __call__(self, i=1):
+        self.w.fill_(i & 0xFF)
+        torch.sum(self.r, dim=0, out=self.acc)
 
 
 def kernel_source_sha(name: str) -> str:
@@ -267,6 +331,144 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def capture(path, calls):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for n in calls:
+            path.call(n)
+    return g
+
+
+def time_segments(path, steps, warmup, flush, dist, device):
+    """Every segment captured once in its own CUDA graph; per step each timed
+    segment is replayed between two CUDA events after an L2 flush, the
+    stand-in segments are replayed without events.  Returns per-segment
+    event times [steps] and the per-step sums."""
+    segs = path.segments()
+    graphs = [capture(path, calls) for _, calls, _ in segs]
+    for _ in range(max(warmup, 0)):
+        for (name, _, timed), g in zip(segs, graphs):
+            if timed:
+                flush()
+            g.replay()
+    torch.cuda.synchronize(device)
+    path.api.check_status(path.status)
+    timed_names = [name for name, _, timed in segs if timed]
+    evs = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)] for n in timed_names}
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    for i in range(steps):
+        for (name, _, timed), g in zip(segs, graphs):
+            if timed:
+                flush(i)
+                evs[name][i][0].record()
+                g.replay()
+                evs[name][i][1].record()
+            else:
+                g.replay()
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    path.api.check_status(path.status)
+    per_seg = {n: [a.elapsed_time(b) for a, b in evs[n]] for n in timed_names}
+    step_ms = [sum(per_seg[n][i] for n in timed_names) for i in range(steps)]
+    del graphs
+    return per_seg, step_ms
+
+
+def time_kernels(path, steps, warmup, flush, dist, device):
+    """Eager launches, one at a time: before each dispatch/combine launch an L2
+    flush, then CUDA events around the launch alone (the stand-in launches
+    run between them, untimed).  Returns {launch: [ms per step]}."""
+    names = path.launches()
+    for _ in range(max(warmup, 0)):
+        for n in names:
+            if n in METHOD:
+                flush()
+            path.call(n)
+    torch.cuda.synchronize(device)
+    evs = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)] for n in names if n in METHOD}
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    for i in range(steps):
+        for n in names:
+            if n in METHOD:
+                flush(i)
+                evs[n][i][0].record()
+                path.call(n)
+                evs[n][i][1].record()
+            else:
+                path.call(n)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    path.api.check_status(path.status)
+    return {n: [a.elapsed_time(b) for a, b in v] for n, v in evs.items()}
+
+
+def time_full_step(path, steps, warmup, flush, dist, device):
+    """The whole path, stand-in included, captured in one graph; one flush
+    per step outside the events."""
+    g = capture(path, path.launches())
+    for _ in range(max(warmup, 0)):
+        flush()
+        g.replay()
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    for i in range(steps):
+        flush(i)
+        evs[i][0].record()
+        g.replay()
+        evs[i][1].record()
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    path.api.check_status(path.status)
+    del g
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def measure_workload(cfg, inp, steps, warmup, dist, device, flush, ws, peak):
+    """Dispatch + combine of one workload: graph-timed segments (the value),
+    eager per-kernel times (the roofline), algorithmic bytes."""
+    path = Path(inp, cfg, device)
+    path.step()                       # first calls: per-device launch caches, outside capture
+    torch.cuda.synchronize(device)
+    per_seg, step_ms = time_segments(path, steps, warmup, flush, dist, device)
+    value, total_max = aggregate_throughput(dist, cfg.T, steps, sum(step_ms), device)
+    ms_per_step = total_max / steps
+    per_kernel = time_kernels(path, steps, warmup, flush, dist, device)
+    N_pad = int(path.lay.expert_offsets[-1].item())
+    nbytes = algorithmic_bytes(cfg.T, cfg.H, cfg.K, cfg.E, cfg.R, path.N, N_pad)
+    method = path.method_launches()
+    step_bytes = sum(nbytes[n] for n in method)
+    mean_k = {n: statistics.fmean(per_kernel[n]) for n in method}
+    total_k = sum(sum(per_kernel[n]) for n in method)
+    kernels = {}
+    for n in method:
+        gbs = nbytes[n] / (mean_k[n] / 1e3) / 1e9
+        kernels[n] = {"function": KERNEL_FUNCTION[n], "mean_ms": mean_k[n],
+                      "share": sum(per_kernel[n]) / total_k, "gbs": gbs, "frac": gbs / peak,
+                      "bytes_per_launch": nbytes[n], "traffic": ncu_traffic(n, cfg.name)}
+    dom = max(method, key=lambda n: sum(per_kernel[n]))
+    gbs = step_bytes / (ms_per_step / 1e3) / 1e9
+    res = {
+        "value": value, "unit": "tokens/s", "ms_per_step": ms_per_step,
+        "p50_ms_per_step": statistics.median(step_ms),
+        "segments_ms": {n: statistics.fmean(v) for n, v in per_seg.items()},
+        "hbm": {"achieved_gbs": gbs, "bytes_per_step": step_bytes, "peak_gbs": peak,
+                "frac": gbs / peak},
+        "dominant": {"kernel": dom, "function": KERNEL_FUNCTION[dom],
+                     "frac": kernels[dom]["frac"], "gbs": kernels[dom]["gbs"]},
+        "kernels": kernels,
+        "N_cap": path.N, "N_pad": N_pad,
+        "launches_per_step": len(path.launches()), "timed_launches_per_step": len(method),
+    }
+    return path, res, nbytes
+
+
 def run_ours(args, cfg, inp, dist, rank, ws, device):
     from combine_moe_dispatch_03_b200 import build as _b
     if rank == 0:
@@ -274,171 +476,106 @@ def run_ours(args, cfg, inp, dist, rank, ws, device):
     if dist is not None:
         dist.barrier()
     _b.build()
-    path = Path(inp, cfg, device)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
-    stream = torch.cuda.current_stream(device)
-
-    for _ in range(max(args.warmup, 0)):
-        flush.fill_(1)
-        path.step()
-    torch.cuda.synchronize(device)
-    path.api.check_status(path.status)
-
-    nk = len(Path.names) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk)] for _ in range(args.steps)]
+    flush = Flush(device)
+    peak, peak_kind = measured_peak()
     sampler = ClockSampler(device.index)
-    barrier(dist, device)
-    torch.cuda.synchronize(device)
     sampler.start()
     time.sleep(0.3)
     t_wall = time.perf_counter()
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        path.step(evs[i])
-    torch.cuda.synchronize(device)
+    path, main, nbytes = measure_workload(cfg, inp, args.steps, args.warmup, dist, device, flush,
+                                          ws, peak)
     t_wall = time.perf_counter() - t_wall
-    barrier(dist, device)
-    path.api.check_status(path.status)
-    # ---- the same step replayed from one CUDA graph (the headline) ----
-    graph = None if args.no_graph else run_graph(args, path, cfg, dist, device, flush)
+    full = None
+    if not args.no_full_step:
+        fms = time_full_step(path, args.steps, args.warmup, flush, dist, device)
+        fv, fmax = aggregate_throughput(dist, cfg.T, args.steps, sum(fms), device)
+        full = {"value": fv, "unit": "tokens/s", "ms_per_step": fmax / args.steps,
+                "launches_per_step": len(path.launches()),
+                "how": "all launches of the step, stand-in included, in one CUDA graph; "
+                       "one L2 flush per step outside the events"}
+    e2e = None if args.no_e2e else run_e2e(args, path, inp, dist, device)
+    del path
+    torch.cuda.empty_cache()
+
+    workloads = {}
+    from combine_moe_dispatch_03_b200.inputs import CONFIGS, make_inputs
+    extra = [] if args.workloads in ("", "none") else args.workloads.split(",")
+    for name in extra:
+        if name == cfg.name:
+            continue
+        wcfg = CONFIGS[name]
+        winp = make_inputs(wcfg, seed=wcfg.seed + rank, with_grad=wcfg.backward)
+        wpath, wres, _ = measure_workload(wcfg, winp, args.steps, args.warmup, dist, device,
+                                          flush, ws, peak)
+        wres["workload"] = wcfg.description
+        wres["timed"] = ("layout+permute | combine + combine backward | dispatch backward"
+                         if wcfg.backward else "layout+permute | combine")
+        workloads[name] = wres
+        del wpath, winp
+        torch.cuda.empty_cache()
     clocks = sampler.stop()
 
-    per_kernel = {n: [] for n in Path.names}
-    step_ms = []
-    for e in evs:
-        for j, n in enumerate(Path.names):
-            per_kernel[n].append(e[j].elapsed_time(e[j + 1]))
-        step_ms.append(e[0].elapsed_time(e[-1]))
-    total_ms = sum(step_ms)
-    eager_value, total_ms_max = aggregate_throughput(dist, cfg.T, args.steps, total_ms, device)
-    eager = {"value": eager_value, "unit": "tokens/s", "ms_per_step": total_ms_max / args.steps,
-             "p50_ms_per_step": statistics.median(step_ms), "steps": args.steps,
-             "how": "seven eager launches per step, a CUDA event between every two"}
-    main = graph if graph is not None else eager
-    value, ms_per_step = main["value"], main["ms_per_step"]
-
-    N_pad = int(path.lay.expert_offsets[-1].item())
-    nbytes = algorithmic_bytes(cfg.T, cfg.H, cfg.K, cfg.E, cfg.R, path.N, N_pad)
-    step_bytes = sum(nbytes.values())
-    mean_k = {n: statistics.fmean(v) for n, v in per_kernel.items()}
-    share = {n: sum(v) / total_ms for n, v in per_kernel.items()}
-    # The dominant kernel is the kernel FUNCTION with the largest share of the
-    # step: launches of the same kernel (the stand-in runs forward and
-    # backward; combine runs weighted and unit-weight) are pooled.
-    funcs = {}
-    for n in Path.names:
-        funcs.setdefault(KERNEL_FUNCTION[n], []).append(n)
-    dom_fn = max(funcs, key=lambda f: sum(sum(per_kernel[n]) for n in funcs[f]))
-    members = funcs[dom_fn]
-    dom = members[0]
-    dom_launches = sum(len(per_kernel[n]) for n in members)
-    dom_mean_ms = sum(sum(per_kernel[n]) for n in members) / dom_launches
-    dom_bytes = sum(nbytes[n] * len(per_kernel[n]) for n in members) / dom_launches
-    peak, peak_kind = measured_peak()
-    achieved = dom_bytes / (dom_mean_ms / 1e3) / 1e9
-    hbm_gbs = step_bytes / (ms_per_step / 1e3) / 1e9
-
-    # ---- end to end: pinned host inputs -> device -> step -> host results ----
-    e2e = None if args.no_e2e else run_e2e(args, path, inp, dist, device, flush)
-
+    k = main["kernels"]
+    dom = main["dominant"]["kernel"]
     result = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "p50_ms_per_step": main["p50_ms_per_step"], "timing": main["how"],
-        "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "metric": METRIC, "value": main["value"], "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
+        "p50_ms_per_step": main["p50_ms_per_step"],
+        "timing": "dispatch and combine segments, each captured in its own CUDA graph and "
+                  "replayed per step between CUDA events; the stand-in expert runs between "
+                  "them outside the events",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
         "config": {
             "workload": cfg.description, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K,
-            "R": cfg.R, "align": cfg.align, "N_cap": path.N, "N_pad": N_pad,
+            "R": cfg.R, "align": cfg.align, "N_cap": main["N_cap"], "N_pad": main["N_pad"],
             "router_dtype": "fp32", "global_batch": cfg.T * ws, "parallelism": "replicas",
-            "l2": "flushed: 256 MiB device write between timed steps (outside the events)",
-            "step": "layout, permute, stand-in experts, combine, combine backward, "
-                    "stand-in backward, dispatch backward (unit-weight combine)",
+            "l2": "flushed before every timed segment and every timed kernel: 256 MiB device "
+                  "write + 256 MiB read of another buffer, outside the events",
+            "timed": ("layout+permute | combine + combine backward | dispatch backward"
+                      if cfg.backward else "layout+permute | combine"),
+            "untimed": "stand-in expert y = x*s_e (and its backward) between the segments",
         },
-        "hbm": {"achieved_gbs": hbm_gbs, "bytes_per_step": step_bytes, "peak_gbs": peak,
-                "frac": hbm_gbs / peak, "peak_kind": peak_kind},
-        "roofline": {"bound": "hbm", "kernel": dom_fn, "launches": members,
-                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": ncu_traffic(dom, cfg.name), "bytes_per_launch": dom_bytes,
-                     "mean_ms": dom_mean_ms, "peak_kind": peak_kind},
-        "kernels": {n: {"mean_ms": mean_k[n], "share": share[n],
-                        "gbs": nbytes[n] / (mean_k[n] / 1e3) / 1e9,
-                        "frac": nbytes[n] / (mean_k[n] / 1e3) / 1e9 / peak,
-                        "bytes_per_launch": nbytes[n],
-                        "traffic": ncu_traffic(n, cfg.name)} for n in Path.names},
-        "eager": eager,
+        "segments_ms": main["segments_ms"],
+        "hbm": dict(main["hbm"], peak_kind=peak_kind),
+        "roofline": {"bound": "hbm", "kernel": k[dom]["function"], "launch": dom,
+                     "achieved": k[dom]["gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": k[dom]["frac"], "traffic": k[dom]["traffic"],
+                     "bytes_per_launch": k[dom]["bytes_per_launch"], "mean_ms": k[dom]["mean_ms"],
+                     "peak_kind": peak_kind},
+        "kernels": k,
+        "workloads": workloads,
+        "full_step": full,
         "e2e": e2e,
-        "gpu_launches": Path.kernels_per_step * args.steps,
+        "gpu_launches": main["launches_per_step"] * args.steps,
+        "gpu_launches_timed": main["timed_launches_per_step"] * args.steps,
         "clocks": clocks,
-        "wall_s_timed_region": t_wall,
+        "wall_s_headline": t_wall,
     }
     return result
 
 
-def run_graph(args, path, cfg, dist, device, flush):
-    """The step captured once into a CUDA graph (every call only enqueues
-    work on the current stream and allocates nothing, so the seven launches
-    and the layout's memset are capturable) and replayed: same L2 flush
-    between steps, outside the events; per-step CUDA events around each
-    replay on the replaying stream."""
-    graph = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream(device)
-    side.wait_stream(torch.cuda.current_stream(device))
-    with torch.cuda.stream(side):
-        path.step()
-    torch.cuda.current_stream(device).wait_stream(side)
-    torch.cuda.synchronize(device)
-    with torch.cuda.graph(graph):
-        path.step()
-    for _ in range(max(args.warmup, 0)):
-        flush.fill_(1)
-        graph.replay()
-    torch.cuda.synchronize(device)
-    path.api.check_status(path.status)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    barrier(dist, device)
-    torch.cuda.synchronize(device)
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        evs[i][0].record()
-        graph.replay()
-        evs[i][1].record()
-    torch.cuda.synchronize(device)
-    barrier(dist, device)
-    path.api.check_status(path.status)
-    ms = [a.elapsed_time(b) for a, b in evs]
-    value, total_max = aggregate_throughput(dist, cfg.T, args.steps, sum(ms), device)
-    del graph
-    return {"value": value, "unit": "tokens/s", "ms_per_step": total_max / args.steps,
-            "p50_ms_per_step": statistics.median(ms), "steps": args.steps,
-            "how": "one step captured in a CUDA graph, replayed once per timed step"}
-
-
-def run_e2e(args, path, inp, dist, device, flush):
-    """Same metric through pinned host buffers: every step copies its inputs
-    host->device and its results (out, grad_x, grad_w) device->host, inside
-    the timed region.  The steps are pipelined the way a serving loop runs
-    them: step i+1's inputs copy in on one stream and step i-1's results copy
-    out on another while step i computes, with double-buffered device inputs
-    and outputs (events order every reuse).  L2 is not flushed here: every
-    step streams ~5 GB and its inputs alone (134 MB) exceed L2."""
+def run_e2e(args, path, inp, dist, device):
+    """The full step through pinned host buffers: every step copies its
+    inputs host->device and its results (out, and for fwd+bwd grad_x and
+    grad_w) device->host, inside the timed region.  The steps are pipelined
+    the way a serving loop runs them: step i+1's inputs copy in on one stream
+    and step i-1's results copy out on another while step i computes, with
+    double-buffered device inputs and outputs (events order every reuse).
+    L2 is not flushed here: every step's inputs alone exceed L2."""
     steps = max(3, min(args.steps, 50))
-    names_in = ("x", "topk_idx", "weights", "scales", "grad_out")
+    names_in = ["x", "topk_idx", "weights", "scales"] + (["grad_out"] if path.backward else [])
+    attr_in = {"x": "x", "topk_idx": "topk", "weights": "w", "scales": "s", "grad_out": "g"}
+    attr_in = {n: attr_in[n] for n in names_in}
+    attr_out = ("out", "grad_x", "grad_w") if path.backward else ("out",)
     host_in = {k: inp[k].pin_memory() for k in names_in}
-    host_out = {"out": torch.empty_like(path.out, device="cpu").pin_memory(),
-                "grad_x": torch.empty_like(path.grad_x, device="cpu").pin_memory(),
-                "grad_w": torch.empty_like(path.grad_w, device="cpu").pin_memory()}
+    host_out = {a: torch.empty_like(getattr(path, a), device="cpu").pin_memory() for a in attr_out}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    attr_in = {"x": "x", "topk_idx": "topk", "weights": "w", "scales": "s", "grad_out": "g"}
-    attr_out = ("out", "grad_x", "grad_w")
     slots = []
     for k in range(2):
         slot = {}
-        for n, a in attr_in.items():
-            slot[a] = getattr(path, a) if k == 0 else torch.empty_like(getattr(path, a))
-        for a in attr_out:
+        for a in list(attr_in.values()) + list(attr_out):
             slot[a] = getattr(path, a) if k == 0 else torch.empty_like(getattr(path, a))
         slots.append(slot)
     s_in = torch.cuda.Stream(device)
@@ -500,90 +637,141 @@ def run_e2e(args, path, inp, dist, device, flush):
     torch.cuda.synchronize(device)
     for a, t in slots[0].items():       # leave the path on its own buffers
         setattr(path, a, t)
+    path.api.check_status(path.status)
     total = t0.elapsed_time(t1)
     value, total = aggregate_throughput(dist, path.cfg.T, steps, total, device)
     return {"value": value, "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": total / steps,
+            "how": "full step (stand-in included) through the public API; inputs copied in "
+                   "from pinned host memory and results copied out every step",
             "pipelined": "copy-in of step i+1 and copy-out of step i-1 overlap step i (3 streams)"}
 
 
 # ------------------------------------------------------ CPU oracle timing ---
 
-def oracle_step(orc, sample):
-    """One pass of the whole path through the CPU oracle (single thread)."""
-    s = sample
-    lay = orc.layout(s["topk"], s["E"], s["R"], s["align"])
-    pm = orc.permute(s["x"], s["topk"], s["E"], lay["expert_offsets"], s["N"])
-    y = orc.expert_scale(pm["x_perm"], lay["expert_offsets"], lay["tokens_per_expert"], s["s"])
-    orc.combine(y, pm["flat_to_row"], s["w"], seq=False)
-    bw = orc.combine_backward(s["g"], y, pm["row_to_flat"], pm["flat_to_row"], s["w"],
-                              lay["expert_offsets"])
-    gxp = orc.expert_scale(bw["grad_rows"], lay["expert_offsets"], lay["tokens_per_expert"], s["s"])
-    orc.combine(gxp, pm["flat_to_row"], None, seq=False)
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.lower().startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
 
 
-def oracle_sample(cfg, inp, tokens):
+def oracle_prepare(orc, cfg, inp, tokens):
+    """A token sample of the workload plus the stand-in's outputs, which the
+    timed oracle pass takes as inputs (the stand-in is not timed)."""
     from combine_moe_dispatch_03_b200.inputs import bf16_bits
     T = min(tokens, cfg.T)
     T -= T % cfg.R
-    return dict(x=bf16_bits(inp["x"][:T]), topk=inp["topk_idx"][:T].numpy(),
-                w=inp["weights"][:T].numpy(), s=inp["scales"].numpy(),
-                g=bf16_bits(inp["grad_out"][:T]), E=cfg.E, R=cfg.R, align=cfg.align, T=T,
-                N=T * cfg.K + cfg.E * (cfg.align - 1))
+    T = max(T, cfg.R)
+    s = dict(x=bf16_bits(inp["x"][:T]), topk=inp["topk_idx"][:T].numpy(),
+             w=inp["weights"][:T].numpy(), sc=inp["scales"].numpy(), E=cfg.E, R=cfg.R,
+             align=cfg.align, T=T, N=T * cfg.K + cfg.E * (cfg.align - 1), backward=cfg.backward)
+    lay = orc.layout(s["topk"], s["E"], s["R"], s["align"])
+    pm = orc.permute(s["x"], s["topk"], s["E"], lay["expert_offsets"], s["N"])
+    s["y"] = orc.expert_scale(pm["x_perm"], lay["expert_offsets"], lay["tokens_per_expert"],
+                              s["sc"])
+    if cfg.backward:
+        s["g"] = bf16_bits(inp["grad_out"][:T])
+        bw = orc.combine_backward(s["g"], s["y"], pm["row_to_flat"], pm["flat_to_row"], s["w"],
+                                  lay["expert_offsets"])
+        s["gxp"] = orc.expert_scale(bw["grad_rows"], lay["expert_offsets"],
+                                    lay["tokens_per_expert"], s["sc"])
+    return s
 
 
-def time_oracle(cfg, inp, min_s=10.0, max_s=30.0, tokens=1024):
-    import oracle as orc
-    orc.build()
-    sample = oracle_sample(cfg, inp, tokens)
-    oracle_step(orc, sample)   # warm (page-in)
+def oracle_pass(orc, s):
+    """One pass of the timed dispatch + combine steps through the oracle."""
+    lay = orc.layout(s["topk"], s["E"], s["R"], s["align"])
+    pm = orc.permute(s["x"], s["topk"], s["E"], lay["expert_offsets"], s["N"])
+    orc.combine(s["y"], pm["flat_to_row"], s["w"], seq=False)
+    if s["backward"]:
+        orc.combine_backward(s["g"], s["y"], pm["row_to_flat"], pm["flat_to_row"], s["w"],
+                             lay["expert_offsets"])
+        orc.combine(s["gxp"], pm["flat_to_row"], None, seq=False)
+
+
+def time_oracle_leg(orc, s, min_s):
+    oracle_pass(orc, s)    # warm (page-in)
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle_step(orc, sample)
+        oracle_pass(orc, s)
         n += 1
         el = time.perf_counter() - t0
-        if el >= min_s or (el >= max_s * 0.5 and n >= 1):
+        if el >= min_s:
             break
-    return {"value": sample["T"] * n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {sample['T']} tokens of the workload (same H, E, K, R, align), "
-                      f"whole fwd+bwd path, {n} passes in {el:.1f} s, single-threaded C"}
+    return s["T"] * n / el, n, el
+
+
+def time_oracle(cfg, inp, min_s=8.0, tokens=1024):
+    import oracle as orc
+    orc.build()
+    orc.build(openmp=True)
+    orc.use_openmp(False)
+    s = oracle_prepare(orc, cfg, inp, tokens)
+    v1, n1, e1 = time_oracle_leg(orc, s, min_s)
+    orc.use_openmp(True)
+    try:
+        threads = orc.threads()
+        vm, nm, em = time_oracle_leg(orc, s, min_s)
+    finally:
+        orc.use_openmp(False)
+    steps = ("layout, permute, combine, combine backward, dispatch backward" if cfg.backward
+             else "layout, permute, combine")
+    sample = (f"first {s['T']} tokens of the workload (same H, E, K, R, align), the timed "
+              f"dispatch/combine steps ({steps}); stand-in outputs precomputed, untimed")
+    return {"value": vm, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": sample + f"; OpenMP build, {nm} passes in {em:.1f} s",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+            "single_core": {"value": v1, "unit": "tokens/s", "cores": 1,
+                            "sample": sample + f"; plain build, {n1} passes in {e1:.1f} s"}}
 
 
 def run_reference(args, cfg, inp, rank, ws):
-    """The CPU oracle timed as the reference arm (rank 0 only)."""
+    """The CPU oracle (OpenMP build, all host cores) timed as the reference
+    arm, rank 0 only."""
     if rank != 0:
         return None
     import oracle as orc
-    orc.build()
+    orc.build(openmp=True)
+    orc.use_openmp(True)
+    threads = orc.threads()
     # size the per-step sample so that warm-up + timed steps take ~2 minutes
-    probe = oracle_sample(cfg, inp, 256)
+    probe = oracle_prepare(orc, cfg, inp, 256)
     t0 = time.perf_counter()
-    oracle_step(orc, probe)
+    oracle_pass(orc, probe)
     per_token = (time.perf_counter() - t0) / probe["T"]
     budget = 120.0 / (args.steps + args.warmup)
     tokens = int(max(cfg.R, min(cfg.T, budget / max(per_token, 1e-9))))
-    sample = oracle_sample(cfg, inp, tokens)
+    s = oracle_prepare(orc, cfg, inp, tokens)
     for _ in range(max(args.warmup, 0)):
-        oracle_step(orc, sample)
+        oracle_pass(orc, s)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle_step(orc, sample)
+        oracle_pass(orc, s)
         times.append(time.perf_counter() - t0)
+    orc.use_openmp(False)
     total = sum(times)
-    value = sample["T"] * args.steps / total
-    desc = (f"first {sample['T']} tokens of the workload per step (same H, E, K, R, align), "
-            "whole fwd+bwd path, single-threaded C oracle")
+    value = s["T"] * args.steps / total
+    steps = ("layout, permute, combine, combine backward, dispatch backward" if cfg.backward
+             else "layout, permute, combine")
+    desc = (f"first {s['T']} tokens of the workload per step (same H, E, K, R, align), "
+            f"the dispatch/combine steps ({steps}), C oracle built with OpenMP on "
+            f"{threads} threads; stand-in outputs precomputed, untimed")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": cfg.description, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K,
-                   "R": cfg.R, "align": cfg.align, "parallelism": "replicas"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": desc},
+                   "R": cfg.R, "align": cfg.align, "parallelism": "replicas",
+                   "sample_tokens": s["T"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": desc, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -594,13 +782,15 @@ def run_reference(args, cfg, inp, rank, ws):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen3")
+    ap.add_argument("--workloads", default="dsv3,dsv3_skew,mixtral",
+                    help="extra workloads timed in the same run ('none' to skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-full-step", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (profiling of smaller cases; must divide by R)")
     args = ap.parse_args()
@@ -617,7 +807,7 @@ def main():
     ws, rank, local = dist_env()
 
     if args.impl == "reference":
-        inp = make_inputs(cfg, with_grad=True)
+        inp = make_inputs(cfg, with_grad=cfg.backward)
         res = run_reference(args, cfg, inp, rank, ws)
         if res is not None:
             print(json.dumps(res), flush=True)
@@ -627,7 +817,7 @@ def main():
     torch.cuda.set_device(device)
     dist = init_dist(ws)
     try:
-        inp = make_inputs(cfg, seed=cfg.seed + rank, with_grad=True)
+        inp = make_inputs(cfg, seed=cfg.seed + rank, with_grad=cfg.backward)
         res = run_ours(args, cfg, inp, dist, rank, ws, device)
         if rank == 0:
             if ws == 1 and not args.no_cpu_baseline:

@@ -42,6 +42,8 @@ SIGNATURES = {
     "moe_worst_case_rows": (ctypes.c_int64, [_I, _I, _I, _I]),
     "moe_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch_layout_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_dispatch_layout_timeout_test": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
+                                              _P, _L, _P]),
     "moe_permute": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _L, _P, _P, _P, _P, _P]),
     "moe_expert_scale": (_I, [_P, _L, _P, _P, _I, _I, _P, _P, _P, _P]),
     "moe_combine_weighted": (_I, [_P, _L, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
@@ -54,6 +56,7 @@ SIGNATURES = {
                                       _P, _P]),
     "moe_scatter_flat_index": (_I, [_P, _L, _I, _I, _P, _P, _P]),
     "moe_segment_labels": (_I, [_P, _I, _I, _L, _P, _P, _P]),
+    "moe_rank_bases": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "moe_permute_to_ranks": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _L, _I, _P, _P, _I, _P,
                                   _P, _P]),
     "moe_combine_from_ranks": (_I, [_P, _I, _L, _P, _P, _I, _P, _I, _I, _I, _I, _P, _P, _P]),

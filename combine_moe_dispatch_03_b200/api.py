@@ -301,6 +301,33 @@ def segment_labels(counts: torch.Tensor, modulo: int, rows: int,
     return lab
 
 
+def rank_bases(all_counts: torch.Tensor, rank: int, align: int = 1,
+               status: torch.Tensor | None = None, out: tuple | None = None):
+    """moe_rank_bases: from the per-expert counts of every source rank
+    (all_counts [R, E] int32, on the device) the row bases of the direct
+    dispatch for `rank`.  Returns (dest_base [E], own_offsets [E/R + 1],
+    own_counts [E/R], max_rows [1]) int32 device tensors."""
+    _require(all_counts, "all_counts", torch.int32, 2)
+    R, E = all_counts.shape
+    if E % R:
+        raise ValueError(f"{E} experts do not split into {R} ranks")
+    dev = all_counts.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    if out is None:
+        out = (torch.empty(E, **i32), torch.empty(E // R + 1, **i32), torch.empty(E // R, **i32),
+               torch.empty(1, **i32))
+    dest_base, own_off, own_cnt, max_rows = out
+    _check_out(dest_base, "dest_base", (E,), torch.int32, dev)
+    _check_out(own_off, "own_offsets", (E // R + 1,), torch.int32, dev)
+    _check_out(own_cnt, "own_counts", (E // R,), torch.int32, dev)
+    _check_out(max_rows, "max_rows", (1,), torch.int32, dev)
+    st = status if status is not None else new_status(dev)
+    rc = lib().moe_rank_bases(_ptr(all_counts), R, E, rank, align, _ptr(dest_base), _ptr(own_off),
+                              _ptr(own_cnt), _ptr(max_rows), _ptr(st), _stream(dev))
+    check_rc(rc, "moe_rank_bases")
+    return dest_base, own_off, own_cnt, max_rows
+
+
 def permute_to_ranks(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout,
                      dest_base: torch.Tensor, dest_table: torch.Tensor, dest_cap: int, rank: int,
                      own_offsets: torch.Tensor, own_counts: torch.Tensor, zero_pad: bool = True,

@@ -95,6 +95,32 @@ int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int
                                      workspace, status, stream));
 }
 
+int moe_dispatch_layout_timeout_test(const int64_t* topk_idx, int T, int K, int E, int R,
+                                     int align, int32_t* tokens_per_expert, int32_t* counts,
+                                     int32_t* splits, int32_t* tokens_per_rank,
+                                     uint8_t* is_token_in_rank, int32_t* expert_offsets,
+                                     void* workspace, int32_t* status, int64_t limit_ns,
+                                     cudaStream_t stream) {
+    NvtxRange range("moe_dispatch_layout_timeout_test");
+    if (limit_ns < 0 || limit_ns > 100000000) return MOE_ERR_INVALID_ARG;   // at most 0.1 s
+    if (!sizes_ok(T, K, E) || R < 1 || R > MOE_MAX_R || E % R || T % R || align < 1)
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)T * K + (int64_t)E * (align - 1) > INT32_MAX) return MOE_ERR_INVALID_ARG;
+    if (!tokens_per_expert || !counts || !splits || !tokens_per_rank || !expert_offsets ||
+        !workspace || !status)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !is_token_in_rank)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, 8) || !aligned(workspace, 16) || !aligned(tokens_per_expert, 4) ||
+        !aligned(counts, 4) || !aligned(splits, 4) || !aligned(tokens_per_rank, 4) ||
+        !aligned(expert_offsets, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    const cudaError_t err = moe::launch_layout_ex(
+        topk_idx, T, K, E, R, align, tokens_per_expert, counts, splits, tokens_per_rank,
+        is_token_in_rank, expert_offsets, workspace, status, stream, 1u, (uint64_t)limit_ns, 1);
+    if (err == cudaErrorNotSupported) return MOE_ERR_INVALID_ARG;
+    return finish(err);
+}
+
 int moe_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
                 const int32_t* expert_offsets, const void* workspace, int zero_pad,
                 int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat, int32_t* flat_to_row,
@@ -268,6 +294,22 @@ int moe_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows, i
     if (!aligned(counts, 4) || !aligned(labels, 8) || !aligned(status, 4))
         return MOE_ERR_INVALID_ARG;
     return finish(moe::launch_segment_labels(counts, n, modulo, rows, labels, status, stream));
+}
+
+int moe_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
+                   int32_t* dest_base, int32_t* own_offsets, int32_t* own_counts,
+                   int32_t* max_rows, int32_t* status, cudaStream_t stream) {
+    NvtxRange range("moe_rank_bases");
+    if (R < 1 || R > MOE_MAX_R || E < 1 || E > MOE_MAX_E || E % R || rank < 0 || rank >= R ||
+        align < 1)
+        return MOE_ERR_INVALID_ARG;
+    if (!all_counts || !dest_base || !own_offsets || !own_counts || !max_rows || !status)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned(all_counts, 4) || !aligned(dest_base, 4) || !aligned(own_offsets, 4) ||
+        !aligned(own_counts, 4) || !aligned(max_rows, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    return finish(moe::launch_rank_bases(all_counts, R, E, rank, align, dest_base, own_offsets,
+                                         own_counts, max_rows, status, stream));
 }
 
 int moe_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int R,

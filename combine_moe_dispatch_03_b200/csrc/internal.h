@@ -92,6 +92,16 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
                           int32_t* expert_offsets, void* workspace, int32_t* status,
                           cudaStream_t stream);
 
+// launch_layout with the grid barrier's target raised by bar_extra arrivals
+// and its wait bounded by bar_limit_ns; require_coop refuses shapes that
+// would run the non-cooperative path (cudaErrorNotSupported).
+cudaError_t launch_layout_ex(const int64_t* topk_idx, int T, int K, int E, int R, int align,
+                             int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                             int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
+                             int32_t* expert_offsets, void* workspace, int32_t* status,
+                             cudaStream_t stream, unsigned bar_extra, uint64_t bar_limit_ns,
+                             int require_coop);
+
 cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
                            const int32_t* expert_offsets, const void* workspace, int zero_pad,
                            int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat,
@@ -140,6 +150,10 @@ cudaError_t launch_combine_from_ranks(const uint16_t* const* rows, int R, int64_
                                       const int32_t* flat_to_row, const int64_t* topk_idx, int E,
                                       const void* weights, int weight_dtype, int T, int K, int H,
                                       uint16_t* out, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
+                              int32_t* dest_base, int32_t* own_offsets, int32_t* own_counts,
+                              int32_t* max_rows, int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows,
                                   int64_t* labels, int32_t* status, cudaStream_t stream);

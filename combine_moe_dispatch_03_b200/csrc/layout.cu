@@ -83,8 +83,8 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 // Grid barrier for a cooperative launch: every CTA adds one arrival to
 // `bar` (zeroed before the launch) and waits until `target` arrivals.  The
-// wait is bounded; returns false if it gave up.
-__device__ bool grid_barrier(unsigned* bar, unsigned target) {
+// wait is bounded by limit_ns of %globaltimer; returns false if it gave up.
+__device__ bool grid_barrier(unsigned* bar, unsigned target, uint64_t limit_ns) {
     __shared__ int ok;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -96,7 +96,7 @@ __device__ bool grid_barrier(unsigned* bar, unsigned target) {
             unsigned v;
             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
             if (v >= target) break;
-            if (global_timer_ns() - t0 > kBarrierLimitNs) { good = 0; break; }
+            if (global_timer_ns() - t0 > limit_ns) { good = 0; break; }
             __nanosleep(64);
         }
         __threadfence();
@@ -223,7 +223,8 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
               Geometry geo, int32_t* __restrict__ tokens_per_expert, int32_t* __restrict__ counts,
               int32_t* __restrict__ splits, int32_t* __restrict__ tokens_per_rank,
               uint8_t* __restrict__ itr, int32_t* __restrict__ offsets, char* __restrict__ ws,
-              WsLayout wl, int32_t* __restrict__ status, int coop, int staged) {
+              WsLayout wl, int32_t* __restrict__ status, int coop, int staged,
+              unsigned bar_extra, uint64_t bar_limit_ns) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int scratch[kLWarps + 1];
     __shared__ int am_last;
@@ -335,7 +336,7 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
 
     if (coop) {
         // ------- cooperative: one barrier, then phase 3 and phase 2 at once ---
-        if (!grid_barrier(counter, gridDim.x)) {
+        if (!grid_barrier(counter, gridDim.x + bar_extra, bar_limit_ns)) {
             if (tid == 0) atomicOr(status, MOE_ST_TIMEOUT);
             return;
         }
@@ -411,6 +412,17 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
                           int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
                           int32_t* expert_offsets, void* workspace, int32_t* status,
                           cudaStream_t stream) {
+    return launch_layout_ex(topk_idx, T, K, E, R, align, tokens_per_expert, counts, splits,
+                            tokens_per_rank, is_token_in_rank, expert_offsets, workspace, status,
+                            stream, 0u, kBarrierLimitNs, 0);
+}
+
+cudaError_t launch_layout_ex(const int64_t* topk_idx, int T, int K, int E, int R, int align,
+                             int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                             int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
+                             int32_t* expert_offsets, void* workspace, int32_t* status,
+                             cudaStream_t stream, unsigned bar_extra, uint64_t bar_limit_ns,
+                             int require_coop) {
     const Geometry geo = layout_geometry(T, K, R);
     const WsLayout wl = workspace_layout(E, R, geo.n_tiles, (int64_t)T * K);
     char* ws = static_cast<char*>(workspace);
@@ -457,6 +469,7 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
         }
         if (dev < 0 || dev >= 64 || coop_ok[dev].load(std::memory_order_relaxed) != 1) coop = 0;
     }
+    if (require_coop && !coop) return cudaErrorNotSupported;
     // With the barrier, phase 2 reads the rows from global memory: no staging.
     const int stg = coop ? 0 : staged;
     if (coop) {
@@ -464,14 +477,15 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
                         (void*)&align, (void*)&geo, (void*)&tokens_per_expert, (void*)&counts,
                         (void*)&splits, (void*)&tokens_per_rank, (void*)&is_token_in_rank,
                         (void*)&expert_offsets, (void*)&ws, (void*)&wl, (void*)&status,
-                        (void*)&coop, (void*)&stg};
+                        (void*)&coop, (void*)&stg, (void*)&bar_extra, (void*)&bar_limit_ns};
         return cudaLaunchCooperativeKernel((const void*)layout_kernel, dim3(grid), dim3(kLThreads),
                                            args, smem, stream);
     }
     layout_kernel<<<grid, kLThreads, smem, stream>>>(topk_idx, T, K, E, R, align, geo,
                                                      tokens_per_expert, counts, splits,
                                                      tokens_per_rank, is_token_in_rank,
-                                                     expert_offsets, ws, wl, status, coop, stg);
+                                                     expert_offsets, ws, wl, status, coop, stg,
+                                                     bar_extra, bar_limit_ns);
     return cudaGetLastError();
 }
 

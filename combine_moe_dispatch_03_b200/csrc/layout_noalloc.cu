@@ -27,7 +27,10 @@ std::mutex g_scratch_mutex;
 void* g_scratch_ptr[64] = {};
 
 // Device address of g_layout_scratch on the current device, looked up once
-// per device (with that device current) and cached.
+// per device (with that device current) and cached for the life of the
+// process.  The address belongs to the device's context at that first
+// call; cudaDeviceReset destroys it, after which this entry point is not
+// supported in the process (documented in the header).
 int scratch_on_current_device(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;

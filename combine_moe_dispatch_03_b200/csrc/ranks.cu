@@ -183,6 +183,72 @@ combine_from_ranks_kernel(const uint4* const* __restrict__ rows, int R, int64_t 
     warp_status_or(status, bad);
 }
 
+// Row bases of the direct dispatch from the per-expert counts of every
+// source rank (all_counts [R][E]): one CTA.  Each thread takes experts e,
+// sums the column over the source ranks (total) and over the ranks before
+// `rank` (before); one CTA scan of the padded totals over all experts gives
+// every group's start, and an owner's groups start at the scan value of its
+// first expert, so
+//   dest_base[e]    = scan[e] - scan[owner(e)*El] + before[e]
+//   own_offsets[el] = scan[rank*El + el] - scan[rank*El]
+//   max_rows        = max over owners r of scan[(r+1)*El] - scan[r*El].
+__global__ void __launch_bounds__(kBlock)
+rank_bases_kernel(const int32_t* __restrict__ all_counts, int R, int E, int rank, int align,
+                  int32_t* __restrict__ dest_base, int32_t* __restrict__ own_off,
+                  int32_t* __restrict__ own_cnt, int32_t* __restrict__ max_rows,
+                  int32_t* __restrict__ status) {
+    __shared__ int scan[MOE_MAX_E + 1];
+    __shared__ int total[MOE_MAX_E];
+    __shared__ int before[MOE_MAX_E];
+    __shared__ int scratch[kWarps + 1];
+    __shared__ int best;
+    const int tid = threadIdx.x;
+    const int El = E / R;
+    pdl_wait();
+    pdl_trigger();
+    int bad = 0;
+    if (tid == 0) best = 0;
+    for (int e = tid; e < E; e += kBlock) {
+        int64_t tot = 0, bef = 0;
+        for (int s = 0; s < R; ++s) {
+            int64_t c = all_counts[(size_t)s * E + e];
+            if (c < 0) {
+                bad |= MOE_ST_COVERAGE;
+                c = 0;
+            }
+            tot += c;
+            if (s < rank) bef += c;
+        }
+        const int64_t padded = (tot + align - 1) / align * align;
+        if (padded > (int64_t)(INT32_MAX / MOE_MAX_E)) bad |= MOE_ST_CAPACITY;
+        total[e] = (int)tot;
+        before[e] = (int)bef;
+        scan[e] = (int)padded;
+    }
+    __syncthreads();
+    const int grand = block_exclusive_scan<MOE_MAX_E / kBlock>(scan, E, scratch);
+    if (tid == 0) scan[E] = grand;
+    __syncthreads();
+    for (int e = tid; e < E; e += kBlock)
+        dest_base[e] = scan[e] - scan[(e / El) * El] + before[e];
+    const int mine = rank * El;
+    for (int el = tid; el <= El; el += kBlock) {
+        own_off[el] = scan[mine + el] - scan[mine];
+        if (el < El) own_cnt[el] = total[mine + el];
+    }
+    for (int r = tid; r < R; r += kBlock) atomicMax(&best, scan[(r + 1) * El] - scan[r * El]);
+    __syncthreads();
+    if (tid == 0) *max_rows = best;
+    warp_status_or(status, bad);
+}
+
+cudaError_t launch_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
+                              int32_t* dest_base, int32_t* own_offsets, int32_t* own_counts,
+                              int32_t* max_rows, int32_t* status, cudaStream_t stream) {
+    return launch_pdl(rank_bases_kernel, dim3(1), dim3(kBlock), 0, stream, all_counts, R, E, rank,
+                      align, dest_base, own_offsets, own_counts, max_rows, status);
+}
+
 cudaError_t launch_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int K,
                                     int E, int R, int H, const int32_t* dest_base,
                                     const void* workspace, uint16_t* const* dest_rows,

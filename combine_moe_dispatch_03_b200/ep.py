@@ -191,46 +191,49 @@ def ep_combine(y_grouped: torch.Tensor, handle: EPHandle, weights: torch.Tensor,
 # between the experts' writes and the combine.
 
 
-def rank_bases(all_counts: torch.Tensor, rank: int, align: int = 1):
-    """From the per-expert counts of every source rank ([ep_size, E], row s =
-    rank s's tokens_per_expert): (dest_base [E] -- the row where `rank`'s
-    rows of expert e start in e's owner's buffer --, own_offsets
-    [E_local + 1] -- the padded group starts in `rank`'s own buffer --,
-    own_counts [E_local] -- the real rows of each of its groups).  Metadata
-    arithmetic on [ep_size, E] integers."""
-    R, E = all_counts.shape
-    El = E // R
-    c = all_counts.to(torch.int64)
-    total = c.sum(dim=0)                                          # rows of e from all ranks
-    padded = ((total + align - 1) // align * align).view(R, El)
-    start = torch.cumsum(padded, dim=1) - padded                  # group starts per owner
-    before = c[:rank].sum(dim=0)                                  # rows of e from earlier ranks
-    dest_base = (start.reshape(E) + before).to(torch.int32)
-    own_offsets = torch.cat([start[rank], padded[rank].sum().view(1)]).to(torch.int32)
-    own_counts = total.view(R, El)[rank].to(torch.int32)
-    return dest_base.contiguous(), own_offsets.contiguous(), own_counts.contiguous()
+def rank_bases(all_counts: torch.Tensor, rank: int, align: int = 1,
+               status: torch.Tensor | None = None):
+    """From the per-expert counts of every source rank ([ep_size, E] int32 on
+    the device, row s = rank s's tokens_per_expert): (dest_base [E] -- the
+    row where `rank`'s rows of expert e start in e's owner's buffer --,
+    own_offsets [E_local + 1] -- the padded group starts in `rank`'s own
+    buffer --, own_counts [E_local] -- the real rows of each of its groups),
+    computed by the library's moe_rank_bases kernel."""
+    dest_base, own_off, own_cnt, _ = api.rank_bases(all_counts.to(torch.int32).contiguous(), rank,
+                                                    align, status=status)
+    return dest_base, own_off, own_cnt
 
 
-def direct_receive_rows(all_counts: torch.Tensor, align: int = 1) -> int:
+def direct_receive_rows(all_counts: torch.Tensor, align: int = 1,
+                        status: torch.Tensor | None = None) -> int:
     """Rows every rank's receive buffer needs for this routing (the largest
-    padded total over the ranks).  One device-to-host copy."""
-    R, E = all_counts.shape
-    total = all_counts.to(torch.int64).sum(dim=0)
-    padded = ((total + align - 1) // align * align).view(R, E // R)
-    return int(padded.sum(dim=1).max().item())
+    padded total over the ranks, from moe_rank_bases).  One device-to-host
+    copy: the host sizes the buffers with it."""
+    _, _, _, max_rows = api.rank_bases(all_counts.to(torch.int32).contiguous(), 0, align,
+                                       status=status)
+    return int(max_rows.item())
 
 
-def direct_plan(tokens_per_expert: torch.Tensor, group=None, align: int = 1):
-    """The metadata of the direct dispatch: ONE all-gather of every rank's
-    per-expert counts [E], then rank_bases for this rank.  Returns
-    (all_counts [ep_size, E], dest_base, own_offsets, own_counts)."""
-    R, rank = dist.get_world_size(group), dist.get_rank(group)
+def gather_counts(tokens_per_expert: torch.Tensor, group=None) -> torch.Tensor:
+    """ONE all-gather of every rank's per-expert counts [E]: all_counts
+    [ep_size, E] int32, row s = rank s's counts."""
+    R = dist.get_world_size(group)
     E = tokens_per_expert.numel()
     all_counts = torch.empty(R, E, dtype=torch.int32, device=tokens_per_expert.device)
     dist.all_gather_into_tensor(all_counts.view(-1),
                                 tokens_per_expert.to(torch.int32).contiguous().view(-1),
                                 group=group)
-    return (all_counts,) + rank_bases(all_counts, rank, align)
+    return all_counts
+
+
+def direct_plan(tokens_per_expert: torch.Tensor, group=None, align: int = 1,
+                status: torch.Tensor | None = None):
+    """The metadata of the direct dispatch: the all-gather of the per-expert
+    counts (gather_counts), then this rank's row bases on the device
+    (rank_bases).  Returns (all_counts [ep_size, E], dest_base, own_offsets,
+    own_counts)."""
+    all_counts = gather_counts(tokens_per_expert, group)
+    return (all_counts,) + rank_bases(all_counts, dist.get_rank(group), align, status)
 
 
 @dataclasses.dataclass
@@ -251,7 +254,7 @@ def ep_dispatch_direct(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int
     rank = dist.get_rank(group)
     st = status if status is not None else api.new_status(x.device)
     lay = api.dispatch_layout(topk_idx, num_experts, 1, 1, status=st)
-    _, dest_base, own_off, own_cnt = direct_plan(lay.tokens_per_expert, group, align)
+    _, dest_base, own_off, own_cnt = direct_plan(lay.tokens_per_expert, group, align, st)
     f2r = api.permute_to_ranks(x, topk_idx, lay, dest_base, dest_table, dest_cap, rank, own_off,
                                own_cnt, status=st)
     return DirectHandle(lay, f2r, own_off, own_cnt, st)

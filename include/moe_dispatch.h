@@ -15,9 +15,10 @@
  * moe_permute_payload (FP8 (data, scales) or any row payload),
  * moe_combine_weighted_f32 / moe_combine_backward_f32 (fp32 rows),
  * moe_scatter_flat_index (the folded restore's scatter), moe_segment_labels
- * (the receive side of expert parallelism across ranks), moe_permute_to_ranks
- * and moe_combine_from_ranks (dispatch into / combine out of the ranks'
- * buffers directly, through peer pointers).
+ * (the receive side of expert parallelism across ranks), moe_rank_bases,
+ * moe_permute_to_ranks and moe_combine_from_ranks (the row bases of, and
+ * dispatch into / combine out of, the ranks' buffers directly, through peer
+ * pointers).
  *
  * Sources (titles of the pages that define the operations):
  *   [DeepEP-272] DeepEP issue "Does Deepep's Dispatch/Combine Support Autograd
@@ -161,6 +162,26 @@ int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int
                         int32_t* expert_offsets, void* workspace, int32_t* status,
                         cudaStream_t stream);
 
+/* TEST ONLY -- not part of the path.  The pages have no counterpart: this
+ * call exists so that a test can watch the layout's bounded grid barrier
+ * give up.  It runs moe_dispatch_layout (same arguments and buffers) with the
+ * barrier's target set one arrival above the number of CTAs, which no launch
+ * can reach, and with the wait bounded by limit_ns nanoseconds (0 to
+ * 100,000,000) instead of 2 s.  Every CTA then waits limit_ns, gives up,
+ * sets MOE_ST_TIMEOUT and returns: the kernel ends after about limit_ns, the
+ * context stays usable, and the outputs written after the barrier
+ * (tokens_per_expert, counts, splits, tokens_per_rank, expert_offsets) are
+ * left untouched; is_token_in_rank and the workspace are written before it.
+ * Errors: as moe_dispatch_layout, plus MOE_ERR_INVALID_ARG for a limit out
+ * of range or for sizes whose layout would not run the cooperative
+ * (barrier) path on this device. */
+int moe_dispatch_layout_timeout_test(const int64_t* topk_idx, int T, int K, int E, int R,
+                                     int align, int32_t* tokens_per_expert, int32_t* counts,
+                                     int32_t* splits, int32_t* tokens_per_rank,
+                                     uint8_t* is_token_in_rank, int32_t* expert_offsets,
+                                     void* workspace, int32_t* status, int64_t limit_ns,
+                                     cudaStream_t stream);
+
 /* moe_dispatch_layout for callers that cannot allocate device memory.  The
  * pages have no counterpart of this call; it exists for callers such as a
  * plugin running inside a server or framework that owns the whole device
@@ -178,7 +199,10 @@ int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int
  *    is enqueued.
  *  - The first call on a device looks up the array's device address (with
  *    that device current) and caches it; make that first call before any
- *    stream capture on the device.
+ *    stream capture on the device.  The cached address belongs to the
+ *    device's context as it was at that first call: after cudaDeviceReset
+ *    (which destroys that context and the library's device array with it)
+ *    this call is not supported in the same process.
  *  - Every call shares the one array, which keeps the last call's contents;
  *    the call clears what must start at zero (a memset of the layout's
  *    counter and accumulators, enqueued on `stream`) and its kernel rewrites
@@ -350,6 +374,37 @@ int moe_scatter_flat_index(const int32_t* row_flat, int64_t N, int T, int K,
  *         misalignment.  One kernel. */
 int moe_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows, int64_t* labels,
                        int32_t* status, cudaStream_t stream);
+
+/* Row bases of expert parallelism without a send buffer ([DS-8190]
+ * Redundancy and Fix: every rank derives where its rows go from the
+ * per-expert counts of all ranks, exchanged once; [DS-AutoEP] Attribution:
+ * group alignment).  The receive buffer of owner rank r holds its experts
+ * [r*El, (r+1)*El) in order, each group padded to a multiple of align, and
+ * inside a group the rows of source rank 0, then 1, ...  From all_counts
+ * [R,E] int32 (row s = tokens_per_expert of source rank s's own tokens):
+ *
+ *   dest_base[e]     = start of e's group in its owner's buffer
+ *                      + sum over s < rank of all_counts[s][e]
+ *   own_offsets[el]  = start of group el in rank `rank`'s own buffer,
+ *   own_offsets[El]  = that buffer's padded total
+ *   own_counts[el]   = sum over s of all_counts[s][rank*El + el]
+ *   max_rows[0]      = the largest padded total over the R owners (the rows
+ *                      every receive buffer needs for this routing)
+ *
+ * The inputs of moe_permute_to_ranks (dest_base, own_offsets, own_counts);
+ * computed on the device, so the only host copy of the plan is the caller's
+ * read of max_rows when it sizes the buffers.
+ * In:  all_counts [R,E] int32 (device).
+ * Out: dest_base [E], own_offsets [E/R + 1], own_counts [E/R], max_rows [1]
+ *      int32 (device).
+ * Status: MOE_ST_COVERAGE for a negative count (counted as 0),
+ *         MOE_ST_CAPACITY if a padded group would overflow int32.
+ * Errors: MOE_ERR_INVALID_ARG for R outside [1, MOE_MAX_R], E outside
+ *         [1, MOE_MAX_E], E % R, rank outside [0, R), align < 1, a null
+ *         pointer or misalignment.  One kernel of one CTA. */
+int moe_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
+                   int32_t* dest_base, int32_t* own_offsets, int32_t* own_counts,
+                   int32_t* max_rows, int32_t* status, cudaStream_t stream);
 
 /* Dispatch straight into the receive buffers of the ranks that own the
  * experts (expert parallelism across GPUs without a send buffer; [DeepEP-272]

@@ -3,9 +3,13 @@
 Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
 leg may import this package.  The product path (the CUDA library and its
 Python binding) never imports, links or executes anything here, and nothing
-here imports the product.  The arithmetic lives in ``moe_oracle.c`` (plain,
-single-threaded C, fp64 where floating point); this module only compiles it
-with gcc, loads it with ctypes and marshals numpy arrays.
+here imports the product.  The arithmetic lives in ``moe_oracle.c`` (plain
+C, fp64 where floating point); this module only compiles it with gcc, loads
+it with ctypes and marshals numpy arrays.  The checker is the plain,
+single-threaded build.  ``use_openmp()`` switches to a second build of the
+same source with ``-fopenmp`` (identical results: its pragmas only split
+independent loop iterations), which the benchmark's multi-core CPU-baseline
+leg times.
 
 Every function cites the passage it follows in ``moe_oracle.c``.  Parity
 status of each function (what pins it) is listed in ``tests/test_oracle_*.py``.
@@ -22,8 +26,10 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "libmoe_oracle.so")
+_LIB_OMP = os.path.join(_HERE, "libmoe_oracle_omp.so")
 _lock = threading.Lock()
-_lib = None
+_libs: dict = {}
+_variant = "plain"
 
 # Status bits of the documented contract (this package's own copy).
 EXPERT_OOR = 1
@@ -32,25 +38,39 @@ ROW_OOR = 4
 COVERAGE = 8
 
 
-def build(force: bool = False) -> str:
+def build(force: bool = False, openmp: bool = False) -> str:
     """Compile moe_oracle.c into libmoe_oracle.so next to it (gcc, -O2, no FMA
-    contraction so every rounding is the one written in the source)."""
-    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
-        return _LIB
-    tmp = _LIB + f".tmp{os.getpid()}"
+    contraction so every rounding is the one written in the source); with
+    ``openmp``, the same source with -fopenmp into libmoe_oracle_omp.so."""
+    out = _LIB_OMP if openmp else _LIB
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(_SRC):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
     cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
-           "-o", tmp, _SRC, "-lm"]
+           *(["-fopenmp"] if openmp else []), "-o", tmp, _SRC, "-lm"]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, _LIB)
-    return _LIB
+    os.replace(tmp, out)
+    return out
+
+
+def use_openmp(on: bool = True) -> None:
+    """Route every function of this module to the OpenMP build (on) or back
+    to the plain single-threaded checker (off)."""
+    global _variant
+    _variant = "openmp" if on else "plain"
+
+
+def threads() -> int:
+    """Threads the current build's loops may use (1 for the plain build)."""
+    return int(_load().oracle_threads())
 
 
 def _load():
-    global _lib
     with _lock:
-        if _lib is not None:
-            return _lib
-        lib = ctypes.CDLL(build())
+        lib = _libs.get(_variant)
+        if lib is not None:
+            return lib
+        lib = ctypes.CDLL(build(openmp=_variant == "openmp"))
         P = ctypes.c_void_p
         I = ctypes.c_int
         L = ctypes.c_int64
@@ -84,7 +104,11 @@ def _load():
         lib.oracle_combine_f32.restype = I
         lib.oracle_combine_backward_f32.argtypes = [P, P, L, P, P, P, I, I, I, P, I, I, P, P]
         lib.oracle_combine_backward_f32.restype = I
-        _lib = lib
+        lib.oracle_rank_bases.argtypes = [P, I, I, I, I, P, P, P, P]
+        lib.oracle_rank_bases.restype = I
+        lib.oracle_threads.argtypes = []
+        lib.oracle_threads.restype = I
+        _libs[_variant] = lib
         return lib
 
 
@@ -144,6 +168,23 @@ def output_splits(topk_idx: np.ndarray, E: int, R: int) -> np.ndarray:
     T, K = topk_idx.shape
     out = np.zeros((R, R), np.int32)
     _load().oracle_output_splits(_p(topk_idx), T, K, E, R, _p(out))
+    return out
+
+
+def rank_bases(all_counts: np.ndarray, rank: int, align: int) -> dict:
+    """Row bases of the direct expert-parallel dispatch from the per-expert
+    counts of every source rank ([R, E]): dest_base [E], own_offsets
+    [E/R + 1], own_counts [E/R], max_rows (see moe_oracle.c)."""
+    all_counts = _c(all_counts, np.int32)
+    R, E = all_counts.shape
+    El = E // R
+    out = dict(dest_base=np.zeros(E, np.int32), own_offsets=np.zeros(El + 1, np.int32),
+               own_counts=np.zeros(El, np.int32))
+    mx = np.zeros(1, np.int32)
+    st = _load().oracle_rank_bases(_p(all_counts), R, E, rank, align, _p(out["dest_base"]),
+                                   _p(out["own_offsets"]), _p(out["own_counts"]), _p(mx))
+    out["max_rows"] = int(mx[0])
+    out["status"] = st
     return out
 
 

@@ -7,8 +7,13 @@
  * CUDA library; the status bit values below are this file's own copy of the
  * documented contract.
  *
- * Every routine is single-threaded, uses plain loops, and does its floating
- * point in fp64 unless a rounding step is part of the definition.  Sources:
+ * Every routine uses plain loops and does its floating point in fp64 unless a
+ * rounding step is part of the definition.  The plain build (no -fopenmp) is
+ * single-threaded and is the checker.  A second build of this same file with
+ * -fopenmp serves only as the multi-core CPU baseline: its pragmas split
+ * loops whose iterations are independent (each writes its own outputs and
+ * the status bits are OR-reduced), so both builds give identical results.
+ * Sources:
  *
  *  [DeepEP-272]  DeepEP issue "Does Deepep's Dispatch/Combine Support Autograd
  *                Like PyTorch's all_to_all?" -- get_dispatch_layout outputs
@@ -46,6 +51,18 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Threads the loops below may use: 1 in the plain build. */
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 /* Status bits (the library's documented values; this file's own copy). */
 #define ORC_EXPERT_OOR 1
@@ -164,6 +181,57 @@ void oracle_output_splits(const int64_t* topk_idx, int T, int K, int E, int R, i
         }
 }
 
+/* Row bases of expert parallelism without a send buffer ([DS-8190]
+ * Redundancy: each source rank s knows its assignments to every expert, and
+ * the matrix of those counts over the ranks fixes where every rank's rows go;
+ * [DS-AutoEP] Attribution: group alignment for the grouped GEMM).  The
+ * receive buffer of owner rank r holds its experts [r*El, (r+1)*El) in
+ * order, each expert's group padded to a multiple of align, and inside a
+ * group the rows of source rank 0 first, then rank 1, and so on.  From
+ * all_counts [R][E] (row s = the per-expert counts of source rank s):
+ *
+ *   own_counts[el]  = sum over s of all_counts[s][rank*El + el]
+ *   own_offsets[el] = padded start of group el in rank `rank`'s buffer,
+ *   own_offsets[El] = that buffer's padded total
+ *   dest_base[e]    = padded start of e's group in its owner's buffer
+ *                     + sum over s < rank of all_counts[s][e]
+ *   max_rows        = the largest padded total over the owners
+ *
+ * Returns ORC_COVERAGE (and treats the count as 0) for a negative count. */
+int oracle_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
+                      int32_t* dest_base, int32_t* own_offsets, int32_t* own_counts,
+                      int32_t* max_rows) {
+    int status = 0;
+    int El = E / R;
+    int64_t best = 0;
+    for (int r = 0; r < R; ++r) {
+        int64_t start = 0;   /* running padded start inside owner r's buffer */
+        for (int el = 0; el < El; ++el) {
+            int e = r * El + el;
+            int64_t total = 0, before = 0;
+            for (int s = 0; s < R; ++s) {
+                int64_t c = all_counts[(int64_t)s * E + e];
+                if (c < 0) {
+                    status |= ORC_COVERAGE;
+                    c = 0;
+                }
+                total += c;
+                if (s < rank) before += c;
+            }
+            dest_base[e] = (int32_t)(start + before);
+            if (r == rank) {
+                own_offsets[el] = (int32_t)start;
+                own_counts[el] = (int32_t)total;
+            }
+            start += ((total + align - 1) / align) * align;
+        }
+        if (r == rank) own_offsets[El] = (int32_t)start;
+        if (start > best) best = start;
+    }
+    *max_rows = (int32_t)best;
+    return status;
+}
+
 /* ------------------------------------------------------------- permute --- */
 
 typedef struct {
@@ -210,6 +278,7 @@ int oracle_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int
     }
     qsort(list, (size_t)n, sizeof(orc_assign), orc_cmp_assign);
 
+#pragma omp parallel for schedule(static)
     for (int64_t row = 0; row < N_cap; ++row) row_to_flat[row] = -1;
     if ((int64_t)offsets[E] > N_cap) status |= ORC_CAPACITY;
 
@@ -233,7 +302,9 @@ int oracle_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int
         i = j;
     }
     if (zero_pad) {
-        for (int64_t row = 0; row < (int64_t)offsets[E] && row < N_cap; ++row)
+        int64_t end = (int64_t)offsets[E] < N_cap ? (int64_t)offsets[E] : N_cap;
+#pragma omp parallel for schedule(static)
+        for (int64_t row = 0; row < end; ++row)
             if (row_to_flat[row] < 0) memset(x_perm + row * H, 0, sizeof(uint16_t) * (size_t)H);
     }
     free(list);
@@ -331,6 +402,7 @@ void oracle_bruteforce_rows(const int64_t* topk_idx, int T, int K, int E, const 
 void oracle_expert_scale(const uint16_t* rows, const int32_t* offsets,
                          const int32_t* tokens_per_expert, int E, int H, const float* scales,
                          uint16_t* out) {
+#pragma omp parallel for schedule(dynamic, 1)
     for (int e = 0; e < E; ++e) {
         int64_t begin = offsets[e];
         int64_t real_end = begin + tokens_per_expert[e];
@@ -365,6 +437,7 @@ void oracle_expert_scale(const uint16_t* rows, const int32_t* offsets,
 int oracle_combine(const uint16_t* rows, int64_t N_cap, const int32_t* flat_to_row,
                    const float* w, int T, int K, int H, double* out_ref, uint16_t* out_seq) {
     int status = 0;
+#pragma omp parallel for reduction(|: status) schedule(static)
     for (int t = 0; t < T; ++t) {
         for (int h = 0; h < H; ++h) {
             double sum = 0.0;
@@ -397,6 +470,7 @@ int oracle_combine(const uint16_t* rows, int64_t N_cap, const int32_t* flat_to_r
 int oracle_combine_f32(const float* rows, int64_t N_cap, const int32_t* flat_to_row,
                        const float* w, int T, int K, int H, double* out_ref, float* out_seq) {
     int status = 0;
+#pragma omp parallel for reduction(|: status) schedule(static)
     for (int t = 0; t < T; ++t) {
         for (int h = 0; h < H; ++h) {
             double sum = 0.0;
@@ -487,6 +561,7 @@ int oracle_combine_backward(const uint16_t* g, const uint16_t* rows, int64_t N_c
                             const float* w, int T, int K, int H, const int32_t* offsets, int E,
                             int zero_pad, uint16_t* grad_rows, double* grad_w) {
     int status = 0;
+#pragma omp parallel for reduction(|: status) schedule(static)
     for (int t = 0; t < T; ++t)
         for (int k = 0; k < K; ++k) {
             int64_t f = (int64_t)t * K + k;
@@ -507,7 +582,9 @@ int oracle_combine_backward(const uint16_t* g, const uint16_t* rows, int64_t N_c
             if (grad_w) grad_w[f] = dot;
         }
     if (zero_pad) {
-        for (int64_t row = 0; row < (int64_t)offsets[E] && row < N_cap; ++row)
+        int64_t end = (int64_t)offsets[E] < N_cap ? (int64_t)offsets[E] : N_cap;
+#pragma omp parallel for schedule(static)
+        for (int64_t row = 0; row < end; ++row)
             if (row_to_flat[row] < 0) memset(grad_rows + row * H, 0, sizeof(uint16_t) * (size_t)H);
     }
     return status;
@@ -525,6 +602,7 @@ int oracle_combine_backward_f32(const float* g, const float* rows, int64_t N_cap
                                 const float* w, int T, int K, int H, const int32_t* offsets,
                                 int E, int zero_pad, float* grad_rows, double* grad_w) {
     int status = 0;
+#pragma omp parallel for reduction(|: status) schedule(static)
     for (int t = 0; t < T; ++t)
         for (int k = 0; k < K; ++k) {
             int64_t f = (int64_t)t * K + k;
@@ -545,7 +623,9 @@ int oracle_combine_backward_f32(const float* g, const float* rows, int64_t N_cap
             if (grad_w) grad_w[f] = dot;
         }
     if (zero_pad) {
-        for (int64_t row = 0; row < (int64_t)offsets[E] && row < N_cap; ++row)
+        int64_t end = (int64_t)offsets[E] < N_cap ? (int64_t)offsets[E] : N_cap;
+#pragma omp parallel for schedule(static)
+        for (int64_t row = 0; row < end; ++row)
             if (row_to_flat[row] < 0) memset(grad_rows + row * H, 0, sizeof(float) * (size_t)H);
     }
     return status;

@@ -1,18 +1,26 @@
 """Dispatch and combine across R ranks, emulated in one process on one GPU.
 
 Every rank's send and receive steps run in the library's kernels (layout,
-permute, segment labels, combine); the exchanges between ranks are plain
-tensor copies of exactly what all_to_all_single would deliver, so no kernel
-waits on another.  Against the single-device path with the ranks as logical
-groups: every rank's plan equals the single-device count matrix and splits,
-the expert-grouped rows of every local expert are bit-identical to that
-expert's rows there (pads zero), and the combined output of every rank's
-tokens is bit-identical to the single-device output."""
+permute, segment labels, rank bases, stand-in expert, combine); the
+exchanges between ranks are plain tensor copies of exactly what
+all_to_all_single would deliver, so no kernel waits on another.  Every
+expected value comes from the CPU oracle with the ranks as logical groups:
+every rank's plan equals the oracle's count matrix and splits; the
+expert-grouped rows of every local expert, and the stand-in expert's output
+rows, are bit-identical to that expert's rows in the oracle's single-device
+buffers (pads zero); the combined output of every rank's tokens is
+bit-identical to the oracle's FP32 slot-order chain and within
+2^-7*|ref| + 1e-6 of its fp64 reference.  (It is also bit-identical to the
+single-device CUDA path.)"""
+import types
+
 import numpy as np
 import pytest
 import torch
 
-from combine_moe_dispatch_03_b200.inputs import CONFIGS, custom_inputs, make_inputs
+import oracle as orc
+from _pipeline import assert_within_tol, f32, to_bits
+from combine_moe_dispatch_03_b200.inputs import CONFIGS, bf16_bits, custom_inputs, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -27,6 +35,39 @@ def _built():
 
 def _i16(t):
     return t.contiguous().view(torch.int16)
+
+
+def _oracle(inp, R, E, align):
+    """The single-device path on the CPU oracle, ranks as logical groups."""
+    x = bf16_bits(inp["x"])
+    topk = inp["topk_idx"].numpy()
+    T, K = topk.shape
+    lay = orc.layout(topk, E, R, align)
+    off = lay["expert_offsets"]
+    pm = orc.permute(x, topk, E, off, int(off[-1]))
+    y = orc.expert_scale(pm["x_perm"], off, lay["tokens_per_expert"], inp["scales"].numpy())
+    cb = orc.combine(y, pm["flat_to_row"], inp["weights"].numpy())
+    assert lay["status"] == 0 and pm["status"] == 0 and cb["status"] == 0
+    return dict(lay=lay, off=off, cnt=lay["tokens_per_expert"], x_perm=pm["x_perm"], y=y,
+                ref=cb["ref"], seq=cb["seq"])
+
+
+def _check_rows(got_bits, want_bits, what):
+    if not np.array_equal(got_bits, want_bits):
+        bad = np.argwhere(got_bits != want_bits)
+        raise AssertionError(f"{what}: {len(bad)} elements differ, first at {tuple(bad[0])}")
+
+
+def _check_out(out_s, orc_ref, s, Tb, what):
+    got = to_bits(out_s)
+    _check_rows(got, orc_ref["seq"][s * Tb:(s + 1) * Tb], what + " vs the oracle's FP32 chain")
+    assert_within_tol(f32(got), orc_ref["ref"][s * Tb:(s + 1) * Tb].astype(np.float32),
+                      what + " vs the oracle's fp64 reference")
+
+
+def _local_layout(off, cnt):
+    """What moe_expert_scale reads of a layout: the groups of one buffer."""
+    return types.SimpleNamespace(expert_offsets=off, tokens_per_expert=cnt, E=cnt.shape[0])
 
 
 @pytest.mark.parametrize("R,E,K,Tb,H,align,skew", [
@@ -60,16 +101,10 @@ def _run_emulated(inp, R, E, align):
     H = inp["x"].shape[1]
     Tb, El = T // R, E // R
     x, w, tk = inp["x"].to(dev), inp["weights"].to(dev), inp["topk_idx"].to(dev)
+    sc = inp["scales"].to(dev)
     st = api.new_status(dev)
-
-    # single device, ranks as logical groups
-    lay = api.dispatch_layout(tk, E, R, align, status=st)
-    xp, _, f2r = api.permute(x, tk, lay, status=st)
-    out_ref = api.combine_weighted(xp * 2, f2r, w, status=st)
-    off = lay.expert_offsets.cpu().tolist()
-    cnt = lay.tokens_per_expert.cpu().tolist()
-    counts_all = lay.counts.cpu()
-    splits_all = lay.splits.cpu()
+    o = _oracle(inp, R, E, align)
+    off, cnt = o["off"], o["cnt"]
 
     # send side of every rank
     sends = [ep.dispatch_send(x[r * Tb:(r + 1) * Tb].contiguous(),
@@ -79,12 +114,13 @@ def _run_emulated(inp, R, E, align):
     for r in range(R):
         received = torch.stack([sends[s][4][r] for s in range(R)]).to(torch.int32).contiguous()
         plans.append(ep.plan_from_counts(sends[r][4].to(torch.int32), received))
-        assert torch.equal(plans[r].received_counts.cpu(), counts_all[:, r, :])
-        assert plans[r].input_splits == splits_all[r, :].tolist()
-        assert plans[r].output_splits == splits_all[:, r].tolist()
+        np.testing.assert_array_equal(plans[r].received_counts.cpu().numpy(),
+                                      o["lay"]["counts"][:, r, :])
+        assert plans[r].input_splits == o["lay"]["splits"][r, :].tolist()
+        assert plans[r].output_splits == o["lay"]["splits"][:, r].tolist()
     # row exchange: rank r receives, source by source, the rows each sends to r
     starts = [np.concatenate([[0], np.cumsum(p.input_splits)]) for p in plans]
-    handles, grouped = [], []
+    handles, ys = [], []
     for r in range(R):
         parts = [sends[s][0][starts[s][r]:starts[s][r + 1]] for s in range(R)]
         recv = torch.cat(parts).contiguous()
@@ -92,23 +128,33 @@ def _run_emulated(inp, R, E, align):
         gr, rlay, rr2f, rf2r = ep.dispatch_recv(recv, plans[r], align, st)
         handles.append(ep.EPHandle(sends[r][1], sends[r][2], sends[r][3], plans[r], rlay, rr2f,
                                    rf2r, st))
-        grouped.append(gr)
-        roff = rlay.expert_offsets.cpu().tolist()
-        for el in range(El):
-            e, c = r * El + el, cnt[r * El + el]
-            assert roff[el + 1] - roff[el] == off[e + 1] - off[e]
-            assert torch.equal(_i16(gr[roff[el]:roff[el] + c]), _i16(xp[off[e]:off[e] + c])), e
-            assert not _i16(gr[roff[el] + c:roff[el + 1]]).any()
-    # experts, then the reverse exchange and the restore on every source rank
-    backs = [ep.combine_send(grouped[r] * 2, handles[r]) for r in range(R)]
+        # the stand-in expert on this rank's local experts
+        y_r = api.expert_scale(gr, rlay, sc[r * El:(r + 1) * El].contiguous(), status=st)
+        ys.append(y_r)
+        roff = rlay.expert_offsets.cpu().numpy()
+        np.testing.assert_array_equal(roff, off[r * El:(r + 1) * El + 1] - off[r * El])
+        n = int(roff[-1])
+        lo = int(off[r * El])
+        _check_rows(to_bits(gr[:n]), o["x_perm"][lo:lo + n], f"rank {r} grouped rows")
+        _check_rows(to_bits(y_r[:n]), o["y"][lo:lo + n], f"rank {r} expert rows")
+    # the reverse exchange and the restore on every source rank
+    backs = [ep.combine_send(ys[r], handles[r]) for r in range(R)]
     rstarts = [np.concatenate([[0], np.cumsum(p.output_splits)]) for p in plans]
+    outs = []
     for s in range(R):
         returned = torch.empty(Tb * K, H, dtype=torch.bfloat16, device=dev)
         parts = torch.cat([backs[r][rstarts[r][s]:rstarts[r][s + 1]] for r in range(R)])
         returned[:parts.shape[0]] = parts
         out_s = ep.combine_recv(returned, handles[s], w[s * Tb:(s + 1) * Tb].contiguous(),
                                 validate=True)
-        assert torch.equal(_i16(out_s), _i16(out_ref[s * Tb:(s + 1) * Tb])), s
+        _check_out(out_s, o, s, Tb, f"rank {s} output")
+        outs.append(out_s)
+    api.check_status(st)
+    # also bit-identical to the single-device CUDA path
+    lay = api.dispatch_layout(tk, E, R, align, status=st)
+    xp, _, f2r = api.permute(x, tk, lay, status=st)
+    out_ref = api.combine_weighted(api.expert_scale(xp, lay, sc, status=st), f2r, w, status=st)
+    assert torch.equal(_i16(torch.cat(outs)), _i16(out_ref))
     api.check_status(st)
 
 
@@ -138,43 +184,53 @@ def test_ep_direct_emulated_full_size():
 def _run_direct(inp, R, E, align):
     """Every rank stores its rows straight into the R receive buffers (a
     table of addresses: separate buffers on this one GPU, peer addresses
-    across GPUs) and gathers the expert outputs straight from them."""
+    across GPUs) and gathers the expert outputs straight from them; the row
+    bases come from the library's moe_rank_bases on the gathered counts."""
     from combine_moe_dispatch_03_b200 import api, ep
     dev = torch.device("cuda:0")
     T, K = inp["topk_idx"].shape
     H = inp["x"].shape[1]
     Tb, El = T // R, E // R
     x, w, tk = inp["x"].to(dev), inp["weights"].to(dev), inp["topk_idx"].to(dev)
+    sc = inp["scales"].to(dev)
     st = api.new_status(dev)
-    lay = api.dispatch_layout(tk, E, R, align, status=st)
-    xp, _, f2r = api.permute(x, tk, lay, status=st)
-    out_ref = api.combine_weighted(xp * 2, f2r, w, status=st)
-    off = lay.expert_offsets.cpu().tolist()
-    cnt = lay.tokens_per_expert.cpu().tolist()
+    o = _oracle(inp, R, E, align)
+    off = o["off"]
 
     blk = lambda t, s: t[s * Tb:(s + 1) * Tb].contiguous()
     lays = [api.dispatch_layout(blk(tk, s), E, 1, 1, status=st) for s in range(R)]
     all_counts = torch.stack([l.tokens_per_expert for l in lays])      # the all-gather
-    cap = ep.direct_receive_rows(all_counts, align)
+    cap = ep.direct_receive_rows(all_counts, align, status=st)
+    assert cap == max(int(off[(r + 1) * El] - off[r * El]) for r in range(R))
     recv = [torch.full((cap, H), 0x3F80, dtype=torch.int16, device=dev).view(torch.bfloat16)
             for _ in range(R)]
     table = torch.tensor([b.data_ptr() for b in recv], dtype=torch.int64, device=dev)
-    f2rs = []
+    f2rs, owns = [], []
     for s in range(R):
-        dest_base, own_off, own_cnt = ep.rank_bases(all_counts, s, align)
+        dest_base, own_off, own_cnt = ep.rank_bases(all_counts, s, align, status=st)
+        owns.append((own_off, own_cnt))
         f2rs.append(api.permute_to_ranks(blk(x, s), blk(tk, s), lays[s], dest_base, table, cap, s,
                                          own_off, own_cnt, status=st))
+    ys = []
     for r in range(R):
-        _, own_off, own_cnt = ep.rank_bases(all_counts, r, align)
-        roff = own_off.cpu().tolist()
-        for el in range(El):
-            e, c = r * El + el, cnt[r * El + el]
-            assert roff[el + 1] - roff[el] == off[e + 1] - off[e]
-            assert torch.equal(_i16(recv[r][roff[el]:roff[el] + c]), _i16(xp[off[e]:off[e] + c])), e
-            assert not _i16(recv[r][roff[el] + c:roff[el + 1]]).any()
-    ys = [b * 2 for b in recv]
+        own_off, own_cnt = owns[r]
+        roff = own_off.cpu().numpy()
+        np.testing.assert_array_equal(roff, off[r * El:(r + 1) * El + 1] - off[r * El])
+        n, lo = int(roff[-1]), int(off[r * El])
+        _check_rows(to_bits(recv[r][:n]), o["x_perm"][lo:lo + n], f"rank {r} receive buffer")
+        y_r = api.expert_scale(recv[r], _local_layout(own_off, own_cnt),
+                               sc[r * El:(r + 1) * El].contiguous(), status=st)
+        _check_rows(to_bits(y_r[:n]), o["y"][lo:lo + n], f"rank {r} expert rows")
+        ys.append(y_r)
     ytab = torch.tensor([y.data_ptr() for y in ys], dtype=torch.int64, device=dev)
+    outs = []
     for s in range(R):
         out_s = api.combine_from_ranks(ytab, cap, H, f2rs[s], blk(tk, s), E, blk(w, s), status=st)
-        assert torch.equal(_i16(out_s), _i16(out_ref[s * Tb:(s + 1) * Tb])), s
+        _check_out(out_s, o, s, Tb, f"rank {s} output")
+        outs.append(out_s)
+    api.check_status(st)
+    lay = api.dispatch_layout(tk, E, R, align, status=st)
+    xp, _, f2r = api.permute(x, tk, lay, status=st)
+    out_ref = api.combine_weighted(api.expert_scale(xp, lay, sc, status=st), f2r, w, status=st)
+    assert torch.equal(_i16(torch.cat(outs)), _i16(out_ref))
     api.check_status(st)

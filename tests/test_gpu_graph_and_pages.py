@@ -4,10 +4,11 @@ chain is capturable; the layout's memset and cooperative launch included).
 (2) At the four shapes of the pages' benchmark table (DeepSpeed PR "AutoEP:
 support combine_impl=fused_weighted_sum with AutoEP+AutoTP folding",
 Benchmark: hidden 6144, top-4 of 128 and top-8 of 256 experts, 8,192 and
-32,768 tokens), the GPU's fused output has the page's error against an fp64
-reference (1.66e-3 relative L2, the rounding of the bf16 output), its score
-gradient stays within the page's FP32 figure (<= 8.7e-8), and the restore
-allocates nothing beyond its outputs."""
+32,768 tokens), the GPU's row maps and expert rows equal the oracle's, the
+fused output has the page's error against an fp64 reference computed by the
+oracle from the oracle's rows (1.66e-3 relative L2, the rounding of the bf16
+output), its score gradient stays within the page's FP32 figure (<= 8.7e-8),
+and the restore allocates nothing beyond its outputs."""
 import os
 
 import numpy as np
@@ -106,11 +107,30 @@ def test_pages_benchmark_shapes_error_and_memory(name):
     assert bwd_peak <= gr.numel() * 2 + gw.numel() * 4 + 1024
 
     T, K = cfg.T, cfg.K
+    # The oracle's row maps of the whole problem (the maps do not depend on
+    # the row contents, so 16-byte dummy rows stand in for x) must equal the
+    # GPU's bit for bit.
+    topk_np = inp["topk_idx"].numpy()
+    olay = orc.layout(topk_np, cfg.E, cfg.R, cfg.align)
+    N = int(olay["expert_offsets"][-1])
+    opm = orc.permute(np.zeros((T, 8), np.uint16), topk_np, cfg.E, olay["expert_offsets"], N)
+    np.testing.assert_array_equal(f2r.cpu().numpy(), opm["flat_to_row"])
     sample = np.arange(T) if T <= 8192 else np.sort(
         np.random.default_rng(7).choice(T, 2048, replace=False))
     n = sample.shape[0]
-    rows_idx = f2r.cpu().numpy()[sample].reshape(-1)
-    ys = to_bits(y[torch.from_numpy(rows_idx).to(dev)])
+    # The stand-in expert's rows of the sampled assignments from the oracle:
+    # token rows in flat order, grouped by expert (stable), scaled by
+    # oracle_expert_scale, put back in flat order.
+    ex = topk_np[sample].reshape(-1)
+    order = np.argsort(ex, kind="stable")
+    cnt = np.bincount(ex, minlength=cfg.E).astype(np.int32)
+    goff = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int32)
+    rows_flat = np.repeat(bf16_bits(inp["x"])[sample], K, axis=0)
+    ys = np.empty_like(rows_flat)
+    ys[order] = orc.expert_scale(rows_flat[order], goff, cnt, inp["scales"].numpy())
+    # ... which the GPU's expert rows at those assignments must equal.
+    rows_idx = opm["flat_to_row"][sample].reshape(-1)
+    np.testing.assert_array_equal(to_bits(y[torch.from_numpy(rows_idx).to(dev)]), ys)
     f2r_s = np.arange(n * K, dtype=np.int32).reshape(n, K)
     ws = inp["weights"].numpy()[sample]
     ref = orc.combine(ys, f2r_s, ws, seq=False)["ref"]

@@ -155,8 +155,9 @@ def _direct_worker(rank, ws, port, align, q):
         topk = _routing("severe", ws)
         mine = topk[rank * TB:(rank + 1) * TB]
         tpe = torch.from_numpy(orc.layout(mine, E, 1, 1)["tokens_per_expert"])
-        all_counts, dest_base, own_off, own_cnt = ep.direct_plan(tpe, align=align)
-        q.put((rank, all_counts.numpy(), dest_base.numpy(), own_off.numpy(), own_cnt.numpy()))
+        all_counts = ep.gather_counts(tpe)          # the one exchange of the direct dispatch
+        rb = orc.rank_bases(all_counts.numpy(), rank, align)
+        q.put((rank, all_counts.numpy(), rb["dest_base"], rb["own_offsets"], rb["own_counts"]))
     finally:
         dist.destroy_process_group()
 
@@ -164,9 +165,11 @@ def _direct_worker(rank, ws, port, align, q):
 @pytest.mark.parametrize("ws,align", [(2, 8), (4, 1)])
 def test_direct_plan_across_processes(ws, align):
     """The direct dispatch's metadata over real processes: one all-gather of
-    the per-expert counts, then each rank's row bases, which must put every
-    assignment at the oracle's single-device row minus the start of its
-    owner rank's block (the owner's padded groups and real rows likewise)."""
+    the per-expert counts (ep.gather_counts), then each rank's row bases from
+    what it received (the oracle's definition here; the device kernel is
+    pinned to it on the GPU), which must put every assignment at the
+    oracle's single-device row minus the start of its owner rank's block
+    (the owner's padded groups and real rows likewise)."""
     import oracle as orc
     orc.build()
     port = _free_port()

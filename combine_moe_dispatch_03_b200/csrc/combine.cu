@@ -142,12 +142,49 @@ combine_kernel(const uint4* __restrict__ rows, int64_t N_cap, const int32_t* __r
 #define MOE_COMBINE_D 4
 #endif
 
-template <typename Tr, int KT, int U, int D, bool VALIDATE>
+// Where a slot's row lives.  A Slot names one slot's row: LocalRows, one
+// expert-grouped buffer, names it by its row index (from flat_to_row; -1
+// for a skipped slot); RankRows, the buffer of the rank that owns the slot's
+// expert (a table of R buffers, peer addresses across GPUs; plain loads),
+// names it by a pointer to the row (nullptr for a skipped slot).
+struct LocalRows {
+    const uint4* rows;
+    using Slot = int;
+    __device__ __forceinline__ static Slot none() { return -1; }
+    __device__ __forceinline__ bool expert_ok(int64_t) const { return true; }
+    __device__ __forceinline__ Slot slot(int64_t, int r, int) const { return r; }
+    __device__ __forceinline__ static bool valid(Slot s) { return s >= 0; }
+    __device__ __forceinline__ const uint4* ptr(Slot s, int n16) const {
+        return rows + (size_t)(s < 0 ? 0 : s) * n16;
+    }
+    __device__ __forceinline__ static Slot shfl(Slot s, int k) { return __shfl_sync(kFull, s, k); }
+};
+struct RankRows {
+    const uint4* const* rows;
+    const int64_t* topk;
+    int E, El;
+    using Slot = const uint4*;
+    __device__ __forceinline__ static Slot none() { return nullptr; }
+    __device__ __forceinline__ bool expert_ok(int64_t f) const {
+        const int64_t e = topk[f];
+        return e >= 0 && e < E;
+    }
+    __device__ __forceinline__ Slot slot(int64_t f, int r, int n16) const {
+        return rows[topk[f] / El] + (size_t)r * n16;
+    }
+    __device__ __forceinline__ static bool valid(Slot s) { return s != nullptr; }
+    __device__ __forceinline__ const uint4* ptr(Slot s, int) const { return s; }
+    __device__ __forceinline__ static Slot shfl(Slot s, int k) {
+        return reinterpret_cast<Slot>(
+            __shfl_sync(kFull, reinterpret_cast<unsigned long long>(s), k));
+    }
+};
+
+template <typename Tr, int KT, int U, int D, bool VALIDATE, typename Src>
 __global__ void __launch_bounds__(kBlock)
-combine_slots_kernel(const uint4* __restrict__ rows, int64_t N_cap,
-                     const int32_t* __restrict__ r2f, const int32_t* __restrict__ f2r,
-                     const void* __restrict__ w, int wdtype, int T, int n16,
-                     uint4* __restrict__ out, int32_t* __restrict__ status) {
+combine_slots_kernel(Src src_rows, int64_t N_cap, const int32_t* __restrict__ r2f,
+                     const int32_t* __restrict__ f2r, const void* __restrict__ w, int wdtype,
+                     int T, int n16, uint4* __restrict__ out, int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     pdl_wait();
     pdl_trigger();
@@ -160,35 +197,35 @@ combine_slots_kernel(const uint4* __restrict__ rows, int64_t N_cap,
          item += (int64_t)gridDim.x * kWarps) {
         const int64_t t = item / chunks;
         const int c = (int)(item - t * chunks);
-        int myrow = -1;
+        // Lane k < KT resolves slot k: its row and its weight.
+        typename Src::Slot myrow = Src::none();
         float myw = 0.f;
         if (lane < KT) {
             const int64_t f = t * KT + lane;
-            int r = f2r[f];
-            if (r < 0 || (int64_t)r >= N_cap) {
+            const int r = f2r[f];
+            if (r < 0 || (int64_t)r >= N_cap || !src_rows.expert_ok(f)) {
                 if (c == 0) bad |= MOE_ST_ROW_OOR;
-                r = -1;
             } else {
                 myw = w ? load_weight(w, wdtype, f) : 1.f;
                 if (VALIDATE && c == 0 && r2f[r] != (int32_t)f) bad |= MOE_ST_COVERAGE;
+                myrow = src_rows.slot(f, r, n16);
             }
-            myrow = r;
         }
-        int rk[KT];
+        typename Src::Slot rk[KT];
         float wk[KT];
 #pragma unroll
         for (int k = 0; k < KT; ++k) {
-            rk[k] = __shfl_sync(kFull, myrow, k);
+            rk[k] = Src::shfl(myrow, k);
             wk[k] = __shfl_sync(kFull, myw, k);
         }
         const int v0 = c * 32 * U + lane;
         uint4 ring[D][U];
 #pragma unroll
         for (int k = 0; k < D && k < KT; ++k) {
-            const uint4* src = rows + (size_t)(rk[k] < 0 ? 0 : rk[k]) * n16;
+            const uint4* src = src_rows.ptr(rk[k], n16);
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                ring[k][u] = (rk[k] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
+                ring[k][u] = (Src::valid(rk[k]) && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
         }
         float acc[U][Tr::kPer];
 #pragma unroll
@@ -198,7 +235,7 @@ combine_slots_kernel(const uint4* __restrict__ rows, int64_t N_cap,
 #pragma unroll
         for (int k = 0; k < KT; ++k) {
             const int slot = k % D;
-            if (rk[k] >= 0) {
+            if (Src::valid(rk[k])) {
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     float y[Tr::kPer];
@@ -209,10 +246,10 @@ combine_slots_kernel(const uint4* __restrict__ rows, int64_t N_cap,
             }
             if (k + D < KT) {
                 const int kn = k + D;
-                const uint4* src = rows + (size_t)(rk[kn] < 0 ? 0 : rk[kn]) * n16;
+                const uint4* src = src_rows.ptr(rk[kn], n16);
 #pragma unroll
                 for (int u = 0; u < U; ++u)
-                    ring[slot][u] = (rk[kn] >= 0 && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
+                    ring[slot][u] = (Src::valid(rk[kn]) && v0 + 32 * u < n16) ? ld_stream(src + v0 + 32 * u) : zero;
             }
         }
         uint4* dst = out + (size_t)t * n16;
@@ -477,24 +514,43 @@ static int grid_tokens_and_rows(int T, int64_t N_cap, bool sweep_rows, int per_s
     return want < 1 ? 1 : (int)want;
 }
 
-#define MOE_SLOTS_ARGS rows, N_cap, r2f, f2r, w, wd, T, n16, out, status
+#define MOE_SLOTS_ARGS src, N_cap, r2f, f2r, w, wd, T, n16, out, status
 
-template <typename Tr, bool V>
-static void launch_slots_t(int K, int grid, cudaStream_t st, const uint4* rows, int64_t N_cap,
+template <typename Tr, bool V, typename Src>
+static void launch_slots_t(int K, int grid, cudaStream_t st, Src src, int64_t N_cap,
                            const int32_t* r2f, const int32_t* f2r, const void* w, int wd, int T,
                            int n16, uint4* out, int32_t* status) {
     constexpr int U = MOE_COMBINE_U, D = MOE_COMBINE_D;
     // Small K: wider chunks keep as many vectors in flight per lane.
     switch (K) {
-        case 1: launch_pdl(combine_slots_kernel<Tr, 1, 4 * U, 1, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
-        case 2: launch_pdl(combine_slots_kernel<Tr, 2, 2 * U, 2, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
-        case 3: launch_pdl(combine_slots_kernel<Tr, 3, U, (D < 3 ? D : 3), V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
-        case 4: launch_pdl(combine_slots_kernel<Tr, 4, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
-        case 5: launch_pdl(combine_slots_kernel<Tr, 5, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
-        case 6: launch_pdl(combine_slots_kernel<Tr, 6, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
-        case 7: launch_pdl(combine_slots_kernel<Tr, 7, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
-        default: launch_pdl(combine_slots_kernel<Tr, 8, U, D, V>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 1: launch_pdl(combine_slots_kernel<Tr, 1, 4 * U, 1, V, Src>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 2: launch_pdl(combine_slots_kernel<Tr, 2, 2 * U, 2, V, Src>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 3: launch_pdl(combine_slots_kernel<Tr, 3, U, (D < 3 ? D : 3), V, Src>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 4: launch_pdl(combine_slots_kernel<Tr, 4, U, D, V, Src>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 5: launch_pdl(combine_slots_kernel<Tr, 5, U, D, V, Src>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 6: launch_pdl(combine_slots_kernel<Tr, 6, U, D, V, Src>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        case 7: launch_pdl(combine_slots_kernel<Tr, 7, U, D, V, Src>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
+        default: launch_pdl(combine_slots_kernel<Tr, 8, U, D, V, Src>, dim3(grid), dim3(kBlock), 0, st, MOE_SLOTS_ARGS); break;
     }
+}
+
+// Grid of the slot-major kernels: one warp per (token, chunk) item, up to
+// MOE_COMBINE_GRID_PER_SM resident CTAs per SM, and with validation enough
+// threads to sweep the rows.
+#ifndef MOE_COMBINE_GRID_PER_SM
+#define MOE_COMBINE_GRID_PER_SM 8
+#endif
+static int slots_grid(int T, int K, int n16, int64_t N_cap, bool validate) {
+    const int u = K == 1 ? 4 * MOE_COMBINE_U : (K == 2 ? 2 * MOE_COMBINE_U : MOE_COMBINE_U);
+    const int chunks = (n16 + 32 * u - 1) / (32 * u);
+    const int64_t items = (int64_t)T * chunks;
+    const int cap = sm_count_current_device() * MOE_COMBINE_GRID_PER_SM;
+    int64_t want = (items + kWarps - 1) / kWarps;
+    if (validate) {
+        const int64_t rw = (N_cap + kBlock - 1) / kBlock;
+        if (rw > want) want = rw;
+    }
+    return (int)(want > cap ? cap : (want < 1 ? 1 : want));
 }
 
 template <typename Tr>
@@ -503,24 +559,13 @@ static cudaError_t launch_combine_rows(const uint4* rows, int64_t N_cap, const i
                                        int n16, int validate, uint4* out, int32_t* status,
                                        cudaStream_t stream) {
     if (K <= 8) {
-        const int u = K == 1 ? 4 * MOE_COMBINE_U : (K == 2 ? 2 * MOE_COMBINE_U : MOE_COMBINE_U);
-        const int chunks = (n16 + 32 * u - 1) / (32 * u);
-        const int64_t items = (int64_t)T * chunks;
-#ifndef MOE_COMBINE_GRID_PER_SM
-#define MOE_COMBINE_GRID_PER_SM 8
-#endif
-        const int cap = sm_count_current_device() * MOE_COMBINE_GRID_PER_SM;
-        int64_t want = (items + kWarps - 1) / kWarps;
-        if (validate) {
-            const int64_t rw = (N_cap + kBlock - 1) / kBlock;
-            if (rw > want) want = rw;
-        }
-        const int grid = (int)(want > cap ? cap : (want < 1 ? 1 : want));
+        const int grid = slots_grid(T, K, n16, N_cap, validate != 0);
+        const LocalRows src{rows};
         if (validate)
-            launch_slots_t<Tr, true>(K, grid, stream, rows, N_cap, r2f, f2r, w, wd, T, n16, out,
+            launch_slots_t<Tr, true>(K, grid, stream, src, N_cap, r2f, f2r, w, wd, T, n16, out,
                                      status);
         else
-            launch_slots_t<Tr, false>(K, grid, stream, rows, N_cap, r2f, f2r, w, wd, T, n16, out,
+            launch_slots_t<Tr, false>(K, grid, stream, src, N_cap, r2f, f2r, w, wd, T, n16, out,
                                       status);
         return cudaGetLastError();
     }
@@ -531,6 +576,21 @@ static cudaError_t launch_combine_rows(const uint4* rows, int64_t N_cap, const i
     else
         launch_combine_t<Tr, false>(K, grid, stream, rows, N_cap, r2f, f2r, w, wd, T, n16, out,
                                     status);
+    return cudaGetLastError();
+}
+
+// The slot-major restore with every slot's row read from the buffer of its
+// expert's rank (K <= 8); the generic kernel in ranks.cu serves larger K.
+cudaError_t launch_combine_slots_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
+                                            const int32_t* flat_to_row, const int64_t* topk_idx,
+                                            int E, const void* weights, int weight_dtype, int T,
+                                            int K, int H, uint16_t* out, int32_t* status,
+                                            cudaStream_t stream) {
+    const int n16 = H / 8;
+    const RankRows src{reinterpret_cast<const uint4* const*>(rows), topk_idx, E, E / R};
+    launch_slots_t<RowBf16, false>(K, slots_grid(T, K, n16, N_cap, false), stream, src, N_cap,
+                                   nullptr, flat_to_row, weights, weight_dtype, T, n16,
+                                   reinterpret_cast<uint4*>(out), status);
     return cudaGetLastError();
 }
 

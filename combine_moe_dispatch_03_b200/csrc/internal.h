@@ -45,12 +45,20 @@ struct Geometry {
 };
 
 // Tile geometry: about one tile per SM of a 148-SM B200 (the layout kernel
-// runs one 1024-thread CTA per tile), at most kMaxTileAssign assignments per
-// tile.  A pure function of the sizes, so the workspace size is known before
-// any device is touched.
+// runs one 1024-thread CTA per tile), at least kMinTileAssign and at most
+// kMaxTileAssign assignments per tile.  A pure function of the sizes, so the
+// workspace size is known before any device is touched.
+constexpr int kMinTileAssign = 512;            // small problems: fewer, fuller tiles
+
 inline Geometry layout_geometry(int T, int K, int R) {
     const int Tb = R > 0 ? T / R : 0;
     int per_block = R > 0 ? 148 / R : 1;          // tiles per source block, <= 148 in all
+    // No more tiles than it takes to give each at least kMinTileAssign
+    // assignments: a small problem then launches fewer CTAs, with fewer
+    // atomics per counter and a cheaper grid barrier (measured: Mixtral-shaped
+    // layout 14.3 -> 12.7 us; unchanged for the large shapes).
+    const int64_t want = ((int64_t)Tb * K + kMinTileAssign - 1) / kMinTileAssign;
+    if (want < per_block) per_block = (int)want;
     if (per_block < 1) per_block = 1;
     int tt = (Tb + per_block - 1) / per_block;
     int cap = kMaxTileAssign / K;
@@ -154,6 +162,12 @@ cudaError_t launch_combine_from_ranks(const uint16_t* const* rows, int R, int64_
 cudaError_t launch_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
                               int32_t* dest_base, int32_t* own_offsets, int32_t* own_counts,
                               int32_t* max_rows, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_combine_slots_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
+                                            const int32_t* flat_to_row, const int64_t* topk_idx,
+                                            int E, const void* weights, int weight_dtype, int T,
+                                            int K, int H, uint16_t* out, int32_t* status,
+                                            cudaStream_t stream);
 
 cudaError_t launch_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows,
                                   int64_t* labels, int32_t* status, cudaStream_t stream);

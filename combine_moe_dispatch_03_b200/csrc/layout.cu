@@ -136,10 +136,16 @@ __device__ RowOut scan_row(int p, int E, int R, const Geometry& geo, int32_t* ti
     }
     const int total = __shfl_sync(kFull, incl, 31);
     int run = incl - local;
+    // Source block of tile jj (tiles of block sb are [sb*tpb, (sb+1)*tpb)),
+    // tracked incrementally instead of divided out per tile.
+    int nb = j0 < j1 ? (j0 + geo.tpb - 1) / geo.tpb * geo.tpb : 0;   // first block start >= j0
     for (int jj = j0; jj < j1; ++jj) {
         const int v = smem_row ? rows[jj] : __ldcg(rowg + jj);
         if (is_expert) rows[jj] = run;
-        if (jj % geo.tpb == 0) bs[jj / geo.tpb] = run;
+        if (jj == nb) {
+            bs[jj / geo.tpb] = run;
+            nb += geo.tpb;
+        }
         run += v;
     }
     __syncwarp();
@@ -216,6 +222,53 @@ __device__ void scan_row_regs(int p, int E, int R, const Geometry& geo, int32_t*
             tokens_per_rank[(size_t)sb * R + r] = bs[sb + 1] - bs[sb];
     }
     __syncwarp();
+}
+
+// Phases 2 and 3 by one CTA (all kLThreads threads), after phase 1 has
+// produced every tile's per-expert counts and per-rank distinct tokens:
+// one warp per row scans it over the tiles (rewriting expert rows as the
+// per-tile stable bases) and sums it per source block; the row totals give
+// tokens_per_expert, the per-expert counts the permute reads and, padded and
+// scanned, the offsets; the block sums of the expert rows give the splits.
+// `mat` holds the rows [E+R][n_tiles] in shared memory when staged (copied
+// back to tile_base at the end), else nullptr (rows read in global memory).
+// `acc_splits` must be zeroed by the caller before a __syncthreads().
+__device__ void phases_2_3_one_cta(int E, int R, int align, const Geometry& geo, int* mat,
+                                   int* bstart, int* ctot, int* acc_splits, int* scratch,
+                                   int32_t* tile_base, int32_t* tile_tpr, int32_t* expert_count,
+                                   int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                                   int32_t* tokens_per_rank, int32_t* offsets) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int El = E / R, n_tiles = geo.n_tiles, nrows = E + R;
+    int* bs = bstart + warp * (R + 1);
+    for (int p = warp; p < nrows; p += kLWarps) {
+        const RowOut o = scan_row(p, E, R, geo, tile_base, tile_tpr,
+                                  mat ? mat + (size_t)p * n_tiles : nullptr, bs, counts,
+                                  tokens_per_rank);
+        if (p < E) {
+            const int r = p / El;
+            for (int sb = lane; sb < R; sb += 32)
+                atomicAdd(&acc_splits[sb * R + r], bs[sb + 1] - bs[sb]);
+            if (lane == 0) {
+                tokens_per_expert[p] = o.total;
+                expert_count[p] = o.total;
+                ctot[p] = o.total;
+            }
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    if (mat) {
+        const int ne = E * n_tiles;
+        for (int q = tid; q < ne; q += kLThreads) tile_base[q] = mat[q];
+    }
+    // phase 3: offsets and splits
+    if (tid < E) ctot[tid] = ((ctot[tid] + align - 1) / align) * align;
+    __syncthreads();
+    const int total = block_exclusive_scan_1024(ctot, E, scratch);
+    if (tid < E) offsets[tid] = ctot[tid];
+    if (tid == 0) offsets[E] = total;
+    for (int q = tid; q < R * R; q += kLThreads) splits[q] = acc_splits[q];
 }
 
 __global__ void __launch_bounds__(kLThreads, 1)
@@ -375,36 +428,10 @@ layout_kernel(const int64_t* __restrict__ topk, int T, int K, int E, int R, int 
             for (int q = tid; q < nr; q += kLThreads) mat[ne + q] = __ldcg(tile_tpr + q);
         }
         __syncthreads();
-        for (int p = warp; p < nrows; p += kLWarps) {
-            const RowOut o = scan_row(p, E, R, geo, tile_base, tile_tpr,
-                                      staged ? mat + (size_t)p * n_tiles : nullptr, bs, counts,
-                                      tokens_per_rank);
-            if (p < E) {
-                const int r = p / El;
-                for (int sb = lane; sb < R; sb += 32)
-                    atomicAdd(&acc_splits[sb * R + r], bs[sb + 1] - bs[sb]);
-                if (lane == 0) {
-                    tokens_per_expert[p] = o.total;
-                    expert_count[p] = o.total;
-                    ctot[p] = o.total;
-                }
-            }
-            __syncwarp();
-        }
-        __syncthreads();
-        if (staged) {
-            const int ne = E * n_tiles;
-            for (int q = tid; q < ne; q += kLThreads) tile_base[q] = mat[q];
-        }
+        phases_2_3_one_cta(E, R, align, geo, staged ? mat : nullptr, bstart, ctot, acc_splits,
+                           scratch, tile_base, tile_tpr, expert_count, tokens_per_expert, counts,
+                           splits, tokens_per_rank, offsets);
     }
-
-    // ------------------------------------ phase 3: offsets and splits ---
-    if (tid < E) ctot[tid] = ((ctot[tid] + align - 1) / align) * align;
-    __syncthreads();
-    const int total = block_exclusive_scan_1024(ctot, E, scratch);
-    if (tid < E) offsets[tid] = ctot[tid];
-    if (tid == 0) offsets[E] = total;
-    for (int q = tid; q < R * R; q += kLThreads) splits[q] = acc_splits[q];
 }
 
 cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int align,

@@ -275,6 +275,11 @@ cudaError_t launch_combine_from_ranks(const uint16_t* const* rows, int R, int64_
                                       const int32_t* flat_to_row, const int64_t* topk_idx, int E,
                                       const void* weights, int weight_dtype, int T, int K, int H,
                                       uint16_t* out, int32_t* status, cudaStream_t stream) {
+    // K <= 8: the slot-major restore of combine.cu (contiguous row chunks,
+    // several in flight per warp) reading each slot from its rank's buffer.
+    if (K <= 8)
+        return launch_combine_slots_from_ranks(rows, R, N_cap, flat_to_row, topk_idx, E, weights,
+                                               weight_dtype, T, K, H, out, status, stream);
     constexpr int U = 2;
     const int sms = sm_count_current_device();
     int64_t grid = ((int64_t)T + kWarps - 1) / kWarps;

@@ -457,6 +457,11 @@ int moe_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int 
  * Out: out [T,H] bf16.
  * Status: MOE_ST_ROW_OOR for a slot whose row or expert is out of range (it
  *         contributes nothing).
+ * No coverage check: the ranks' buffers carry no map from a row back to the
+ * (source rank, token, slot) it holds, so a stale or duplicated flat_to_row
+ * inside [0, N_cap) combines the wrong rows without a status bit.  The
+ * checked form is moe_combine_weighted with validate = 1 over a local
+ * buffer and its row_to_flat (the all-to-all form of expert parallelism).
  * Errors: MOE_ERR_INVALID_ARG as moe_combine_weighted, plus E % R. */
 int moe_combine_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
                            const int32_t* flat_to_row, const int64_t* topk_idx, int E,

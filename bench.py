@@ -77,14 +77,19 @@ FALLBACK_HBM_GBS = 6650.0
 METHOD = ("layout", "permute", "combine", "combine_backward", "dispatch_backward")
 STAND_IN = ("expert_scale", "expert_scale_bwd")
 
-# Step names -> the kernel function each launches (for K <= 8; larger K uses
-# the generic combine_kernel / combine_bwd_kernel).
-KERNEL_FUNCTION = {
-    "layout": "layout_kernel", "permute": "permute_kernel",
-    "expert_scale": "expert_scale_kernel", "expert_scale_bwd": "expert_scale_kernel",
-    "combine": "combine_slots_kernel", "dispatch_backward": "combine_slots_kernel",
-    "combine_backward": "combine_bwd_slots_kernel",
-}
+# Step names -> the kernel function each launches at top_k = K: the permute
+# moves rows with the copy engine at K <= 2; above K = 8 the combines use
+# their any-K kernels.
+def kernel_function(name: str, K: int) -> str:
+    if name == "permute":
+        return "permute_bulk_kernel" if K <= 2 else "permute_kernel"
+    if name in ("combine", "dispatch_backward"):
+        return "combine_slots_kernel" if K <= 8 else "combine_kernel"
+    if name == "combine_backward":
+        return "combine_bwd_slots_kernel" if K <= 8 else "combine_bwd_kernel"
+    if name == "layout":
+        return "layout_kernel"
+    return "expert_scale_kernel"
 
 KERNEL_SOURCES = {
     "layout": "layout.cu", "permute": "permute.cu", "expert_scale": "expert_scale.cu",
@@ -449,7 +454,7 @@ def measure_workload(cfg, inp, steps, warmup, dist, device, flush, ws, peak):
     kernels = {}
     for n in method:
         gbs = nbytes[n] / (mean_k[n] / 1e3) / 1e9
-        kernels[n] = {"function": KERNEL_FUNCTION[n], "mean_ms": mean_k[n],
+        kernels[n] = {"function": kernel_function(n, cfg.K), "mean_ms": mean_k[n],
                       "share": sum(per_kernel[n]) / total_k, "gbs": gbs, "frac": gbs / peak,
                       "bytes_per_launch": nbytes[n], "traffic": ncu_traffic(n, cfg.name)}
     dom = max(method, key=lambda n: sum(per_kernel[n]))
@@ -460,7 +465,7 @@ def measure_workload(cfg, inp, steps, warmup, dist, device, flush, ws, peak):
         "segments_ms": {n: statistics.fmean(v) for n, v in per_seg.items()},
         "hbm": {"achieved_gbs": gbs, "bytes_per_step": step_bytes, "peak_gbs": peak,
                 "frac": gbs / peak},
-        "dominant": {"kernel": dom, "function": KERNEL_FUNCTION[dom],
+        "dominant": {"kernel": dom, "function": kernel_function(dom, cfg.K),
                      "frac": kernels[dom]["frac"], "gbs": kernels[dom]["gbs"]},
         "kernels": kernels,
         "N_cap": path.N, "N_pad": N_pad,

@@ -88,7 +88,7 @@ def kernel_function(name: str, K: int) -> str:
     if name == "combine_backward":
         return "combine_bwd_slots_kernel" if K <= 8 else "combine_bwd_kernel"
     if name == "layout":
-        return "layout_kernel"
+        return "layout_tiles_kernel + layout_rows_kernel"
     return "expert_scale_kernel"
 
 KERNEL_SOURCES = {

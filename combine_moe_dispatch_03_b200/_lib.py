@@ -42,8 +42,6 @@ SIGNATURES = {
     "moe_worst_case_rows": (ctypes.c_int64, [_I, _I, _I, _I]),
     "moe_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch_layout_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
-    "moe_dispatch_layout_timeout_test": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
-                                              _P, _L, _P]),
     "moe_permute": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _L, _P, _P, _P, _P, _P]),
     "moe_expert_scale": (_I, [_P, _L, _P, _P, _I, _I, _P, _P, _P, _P]),
     "moe_combine_weighted": (_I, [_P, _L, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
@@ -57,9 +55,10 @@ SIGNATURES = {
     "moe_scatter_flat_index": (_I, [_P, _L, _I, _I, _P, _P, _P]),
     "moe_segment_labels": (_I, [_P, _I, _I, _L, _P, _P, _P]),
     "moe_rank_bases": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
-    "moe_permute_to_ranks": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _L, _I, _P, _P, _I, _P,
-                                  _P, _P]),
-    "moe_combine_from_ranks": (_I, [_P, _I, _L, _P, _P, _I, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "moe_permute_to_ranks": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _L, _I, _P, _P, _I,
+                                  _P, _P, _P]),
+    "moe_combine_from_ranks": (_I, [_P, _P, _I, _I, _L, _P, _P, _I, _P, _I, _I, _I, _I, _P, _P,
+                                    _P]),
     "moe_strerror": (ctypes.c_char_p, [_I]),
     "moe_status_bit_name": (ctypes.c_char_p, [_I]),
     "moe_version": (ctypes.c_char_p, []),

@@ -331,10 +331,14 @@ def rank_bases(all_counts: torch.Tensor, rank: int, align: int = 1,
 def permute_to_ranks(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout,
                      dest_base: torch.Tensor, dest_table: torch.Tensor, dest_cap: int, rank: int,
                      own_offsets: torch.Tensor, own_counts: torch.Tensor, zero_pad: bool = True,
+                     claims_table: torch.Tensor | None = None,
                      status: torch.Tensor | None = None, out: torch.Tensor | None = None):
     """moe_permute_to_ranks: rows straight into the buffers listed in
-    dest_table (int64 device tensor [R] of buffer addresses).  Returns
-    flat_to_row [T,K] (row in the buffer of each slot's expert rank)."""
+    dest_table (int64 device tensor [R] of buffer addresses).  With
+    claims_table (int64 device tensor [R] of int32 [dest_cap] array
+    addresses) every stored row also records which (rank, token, slot) it
+    holds, for the restore's coverage check.  Returns flat_to_row [T,K] (row
+    in the buffer of each slot's expert rank)."""
     _require(x, "x", torch.bfloat16, 2)
     _require(topk_idx, "topk_idx", torch.int64, 2)
     T, H = x.shape
@@ -352,23 +356,28 @@ def permute_to_ranks(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout,
     _check_out(dest_base, "dest_base", (E,), torch.int32, dev)
     _check_out(own_offsets, "own_offsets", (E // R + 1,), torch.int32, dev)
     _check_out(own_counts, "own_counts", (E // R,), torch.int32, dev)
+    if claims_table is not None:
+        _check_out(claims_table, "claims_table", (R,), torch.int64, dev)
     f2r = out if out is not None else torch.empty(T, K, dtype=torch.int32, device=dev)
     _check_out(f2r, "flat_to_row", (T, K), torch.int32, dev)
     st = status if status is not None else new_status(dev)
     rc = lib().moe_permute_to_ranks(_ptr(x), _ptr(topk_idx), T, K, E, R, H, _ptr(dest_base),
-                                    _ptr(layout.workspace), _ptr(dest_table), dest_cap, rank,
-                                    _ptr(own_offsets), _ptr(own_counts), int(bool(zero_pad)),
-                                    _ptr(f2r), _ptr(st), _stream(dev))
+                                    _ptr(layout.workspace), _ptr(dest_table), _ptr(claims_table),
+                                    dest_cap, rank, _ptr(own_offsets), _ptr(own_counts),
+                                    int(bool(zero_pad)), _ptr(f2r), _ptr(st), _stream(dev))
     check_rc(rc, "moe_permute_to_ranks")
     return f2r
 
 
 def combine_from_ranks(rows_table: torch.Tensor, N_cap: int, H: int, flat_to_row: torch.Tensor,
                        topk_idx: torch.Tensor, num_experts: int, weights: torch.Tensor,
+                       claims_table: torch.Tensor | None = None, rank: int = 0,
                        status: torch.Tensor | None = None, out: torch.Tensor | None = None):
     """moe_combine_from_ranks: fused_weighted_restore reading each slot's row
     from the buffer of its expert's rank (rows_table: int64 device tensor [R]
-    of bf16 [N_cap, H] buffer addresses)."""
+    of bf16 [N_cap, H] buffer addresses).  With claims_table (the one the
+    dispatch filled) and this rank's index, every slot's row is checked to be
+    claimed by this (rank, token, slot): MOE_ST_COVERAGE otherwise."""
     _require(rows_table, "rows_table", torch.int64, 1)
     _require(flat_to_row, "flat_to_row", torch.int32, 2)
     T, K = flat_to_row.shape
@@ -379,8 +388,10 @@ def combine_from_ranks(rows_table: torch.Tensor, N_cap: int, H: int, flat_to_row
     o = out if out is not None else torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     _check_out(o, "out", (T, H), torch.bfloat16, dev)
     st = status if status is not None else new_status(dev)
-    rc = lib().moe_combine_from_ranks(_ptr(rows_table), rows_table.shape[0], N_cap,
-                                      _ptr(flat_to_row), _ptr(topk_idx), num_experts,
+    if claims_table is not None:
+        _check_out(claims_table, "claims_table", (rows_table.shape[0],), torch.int64, dev)
+    rc = lib().moe_combine_from_ranks(_ptr(rows_table), _ptr(claims_table), rows_table.shape[0],
+                                      rank, N_cap, _ptr(flat_to_row), _ptr(topk_idx), num_experts,
                                       _ptr(weights), wd, T, K, H, _ptr(o), _ptr(st), _stream(dev))
     check_rc(rc, "moe_combine_from_ranks")
     return o

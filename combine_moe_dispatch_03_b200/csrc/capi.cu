@@ -95,32 +95,6 @@ int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int
                                      workspace, status, stream));
 }
 
-int moe_dispatch_layout_timeout_test(const int64_t* topk_idx, int T, int K, int E, int R,
-                                     int align, int32_t* tokens_per_expert, int32_t* counts,
-                                     int32_t* splits, int32_t* tokens_per_rank,
-                                     uint8_t* is_token_in_rank, int32_t* expert_offsets,
-                                     void* workspace, int32_t* status, int64_t limit_ns,
-                                     cudaStream_t stream) {
-    NvtxRange range("moe_dispatch_layout_timeout_test");
-    if (limit_ns < 0 || limit_ns > 100000000) return MOE_ERR_INVALID_ARG;   // at most 0.1 s
-    if (!sizes_ok(T, K, E) || R < 1 || R > MOE_MAX_R || E % R || T % R || align < 1)
-        return MOE_ERR_INVALID_ARG;
-    if ((int64_t)T * K + (int64_t)E * (align - 1) > INT32_MAX) return MOE_ERR_INVALID_ARG;
-    if (!tokens_per_expert || !counts || !splits || !tokens_per_rank || !expert_offsets ||
-        !workspace || !status)
-        return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (!topk_idx || !is_token_in_rank)) return MOE_ERR_INVALID_ARG;
-    if (!aligned(topk_idx, 8) || !aligned(workspace, 16) || !aligned(tokens_per_expert, 4) ||
-        !aligned(counts, 4) || !aligned(splits, 4) || !aligned(tokens_per_rank, 4) ||
-        !aligned(expert_offsets, 4) || !aligned(status, 4))
-        return MOE_ERR_INVALID_ARG;
-    const cudaError_t err = moe::launch_layout_ex(
-        topk_idx, T, K, E, R, align, tokens_per_expert, counts, splits, tokens_per_rank,
-        is_token_in_rank, expert_offsets, workspace, status, stream, 1u, (uint64_t)limit_ns, 1);
-    if (err == cudaErrorNotSupported) return MOE_ERR_INVALID_ARG;
-    return finish(err);
-}
-
 int moe_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
                 const int32_t* expert_offsets, const void* workspace, int zero_pad,
                 int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat, int32_t* flat_to_row,
@@ -314,12 +288,16 @@ int moe_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
 
 int moe_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int R,
                          int H, const int32_t* dest_base, const void* workspace,
-                         uint16_t* const* dest_rows, int64_t dest_cap, int rank,
-                         const int32_t* own_offsets, const int32_t* own_counts, int zero_pad,
-                         int32_t* flat_to_row, int32_t* status, cudaStream_t stream) {
+                         uint16_t* const* dest_rows, int32_t* const* dest_claims,
+                         int64_t dest_cap, int rank, const int32_t* own_offsets,
+                         const int32_t* own_counts, int zero_pad, int32_t* flat_to_row,
+                         int32_t* status, cudaStream_t stream) {
     NvtxRange range("moe_permute_to_ranks");
     if (!sizes_ok(T, K, E) || !hidden_ok(H) || R < 1 || R > MOE_MAX_R || E % R || rank < 0 ||
         rank >= R || dest_cap < 0 || dest_cap > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (dest_claims && ((int64_t)T * K > (int64_t(1) << moe::kClaimShift) ||
+                        !aligned(dest_claims, 8)))
         return MOE_ERR_INVALID_ARG;
     if (!dest_base || !workspace || !dest_rows || !own_offsets || !own_counts || !status)
         return MOE_ERR_INVALID_ARG;
@@ -329,17 +307,21 @@ int moe_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int 
         !aligned(own_counts, 4) || !aligned(flat_to_row, 4) || !aligned(status, 4))
         return MOE_ERR_INVALID_ARG;
     return finish(moe::launch_permute_to_ranks(x, topk_idx, T, K, E, R, H, dest_base, workspace,
-                                               dest_rows, dest_cap, rank, own_offsets, own_counts,
-                                               zero_pad, flat_to_row, status, stream));
+                                               dest_rows, dest_claims, dest_cap, rank, own_offsets,
+                                               own_counts, zero_pad, flat_to_row, status, stream));
 }
 
-int moe_combine_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
-                           const int32_t* flat_to_row, const int64_t* topk_idx, int E,
-                           const void* weights, int weight_dtype, int T, int K, int H,
-                           uint16_t* out, int32_t* status, cudaStream_t stream) {
+int moe_combine_from_ranks(const uint16_t* const* rows, const int32_t* const* claims, int R,
+                           int rank, int64_t N_cap, const int32_t* flat_to_row,
+                           const int64_t* topk_idx, int E, const void* weights, int weight_dtype,
+                           int T, int K, int H, uint16_t* out, int32_t* status,
+                           cudaStream_t stream) {
     NvtxRange range("moe_combine_from_ranks");
     if (!sizes_ok(T, K, E) || !hidden_ok(H) || R < 1 || R > MOE_MAX_R || E % R || N_cap < 0 ||
         N_cap > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (claims && (rank < 0 || rank >= R || (int64_t)T * K > (int64_t(1) << moe::kClaimShift) ||
+                   !aligned(claims, 8)))
         return MOE_ERR_INVALID_ARG;
     if (weight_dtype != MOE_DTYPE_F32 && weight_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
     if (!status || !rows) return MOE_ERR_INVALID_ARG;
@@ -349,8 +331,9 @@ int moe_combine_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
         !aligned(weights, wal) || !aligned(out, 16) || !aligned(status, 4))
         return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    return finish(moe::launch_combine_from_ranks(rows, R, N_cap, flat_to_row, topk_idx, E, weights,
-                                                 weight_dtype, T, K, H, out, status, stream));
+    return finish(moe::launch_combine_from_ranks(rows, claims, R, rank, N_cap, flat_to_row,
+                                                 topk_idx, E, weights, weight_dtype, T, K, H, out,
+                                                 status, stream));
 }
 
 const char* moe_strerror(int code) {

@@ -149,7 +149,11 @@ combine_kernel(const uint4* __restrict__ rows, int64_t N_cap, const int32_t* __r
 // names it by a pointer to the row (nullptr for a skipped slot).
 struct LocalRows {
     const uint4* rows;
+    const int32_t* r2f;
     using Slot = int;
+    static constexpr bool kRowSweep = true;
+    // Coverage: the row claims this (token, slot).
+    __device__ __forceinline__ bool check(int64_t f, int r) const { return r2f[r] == (int32_t)f; }
     __device__ __forceinline__ static Slot none() { return -1; }
     __device__ __forceinline__ bool expert_ok(int64_t) const { return true; }
     __device__ __forceinline__ Slot slot(int64_t, int r, int) const { return r; }
@@ -162,8 +166,15 @@ struct LocalRows {
 struct RankRows {
     const uint4* const* rows;
     const int64_t* topk;
-    int E, El;
+    const int32_t* const* claims;   // per rank, the claim of every row
+    int E, El, rank;
     using Slot = const uint4*;
+    // Coverage can only be checked from the slot side: the row in its owner's
+    // buffer must be claimed by this rank's (token, slot).
+    static constexpr bool kRowSweep = false;
+    __device__ __forceinline__ bool check(int64_t f, int r) const {
+        return claims[topk[f] / El][r] == claim_code(rank, f);
+    }
     __device__ __forceinline__ static Slot none() { return nullptr; }
     __device__ __forceinline__ bool expert_ok(int64_t f) const {
         const int64_t e = topk[f];
@@ -207,7 +218,7 @@ combine_slots_kernel(Src src_rows, int64_t N_cap, const int32_t* __restrict__ r2
                 if (c == 0) bad |= MOE_ST_ROW_OOR;
             } else {
                 myw = w ? load_weight(w, wdtype, f) : 1.f;
-                if (VALIDATE && c == 0 && r2f[r] != (int32_t)f) bad |= MOE_ST_COVERAGE;
+                if (VALIDATE && c == 0 && !src_rows.check(f, r)) bad |= MOE_ST_COVERAGE;
                 myrow = src_rows.slot(f, r, n16);
             }
         }
@@ -258,7 +269,7 @@ combine_slots_kernel(Src src_rows, int64_t N_cap, const int32_t* __restrict__ r2
             if (v0 + 32 * u < n16) st_vec(dst + v0 + 32 * u, Tr::pack(acc[u]));
     }
 
-    if (VALIDATE) {
+    if constexpr (VALIDATE && Src::kRowSweep) {
         const int64_t A = (int64_t)T * KT;
         const int64_t stride = (int64_t)gridDim.x * kBlock;
         for (int64_t row = (int64_t)blockIdx.x * kBlock + threadIdx.x; row < N_cap; row += stride) {
@@ -560,7 +571,7 @@ static cudaError_t launch_combine_rows(const uint4* rows, int64_t N_cap, const i
                                        cudaStream_t stream) {
     if (K <= 8) {
         const int grid = slots_grid(T, K, n16, N_cap, validate != 0);
-        const LocalRows src{rows};
+        const LocalRows src{rows, r2f};
         if (validate)
             launch_slots_t<Tr, true>(K, grid, stream, src, N_cap, r2f, f2r, w, wd, T, n16, out,
                                      status);
@@ -581,16 +592,22 @@ static cudaError_t launch_combine_rows(const uint4* rows, int64_t N_cap, const i
 
 // The slot-major restore with every slot's row read from the buffer of its
 // expert's rank (K <= 8); the generic kernel in ranks.cu serves larger K.
-cudaError_t launch_combine_slots_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
-                                            const int32_t* flat_to_row, const int64_t* topk_idx,
-                                            int E, const void* weights, int weight_dtype, int T,
-                                            int K, int H, uint16_t* out, int32_t* status,
-                                            cudaStream_t stream) {
+cudaError_t launch_combine_slots_from_ranks(const uint16_t* const* rows,
+                                            const int32_t* const* claims, int R, int rank,
+                                            int64_t N_cap, const int32_t* flat_to_row,
+                                            const int64_t* topk_idx, int E, const void* weights,
+                                            int weight_dtype, int T, int K, int H, uint16_t* out,
+                                            int32_t* status, cudaStream_t stream) {
     const int n16 = H / 8;
-    const RankRows src{reinterpret_cast<const uint4* const*>(rows), topk_idx, E, E / R};
-    launch_slots_t<RowBf16, false>(K, slots_grid(T, K, n16, N_cap, false), stream, src, N_cap,
-                                   nullptr, flat_to_row, weights, weight_dtype, T, n16,
-                                   reinterpret_cast<uint4*>(out), status);
+    const RankRows src{reinterpret_cast<const uint4* const*>(rows), topk_idx, claims, E, E / R,
+                       rank};
+    const int grid = slots_grid(T, K, n16, N_cap, false);
+    if (claims)
+        launch_slots_t<RowBf16, true>(K, grid, stream, src, N_cap, nullptr, flat_to_row, weights,
+                                      weight_dtype, T, n16, reinterpret_cast<uint4*>(out), status);
+    else
+        launch_slots_t<RowBf16, false>(K, grid, stream, src, N_cap, nullptr, flat_to_row, weights,
+                                       weight_dtype, T, n16, reinterpret_cast<uint4*>(out), status);
     return cudaGetLastError();
 }
 

@@ -101,8 +101,11 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     return v;
 }
 
+// Row stores are never read back by the storing kernel: no L1 allocation
+// (measured: Qwen3-shaped combine + backward 277.2 -> 275.2 us, dispatch
+// 111.7 -> 111.0 us against plain stores; .cs streaming stores about the same).
 __device__ __forceinline__ void st_vec(uint4* p, const uint4& v) {
-    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+    asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
                  "r"(v.z), "r"(v.w)
                  : "memory");
 }
@@ -132,7 +135,7 @@ __device__ __forceinline__ Vec32 ld_stream32(const uint4* p) {
 }
 
 __device__ __forceinline__ void st_vec32(uint4* p, const Vec32& v) {
-    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+    asm volatile("st.global.L1::no_allocate.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
                  "r"(v.lo.x), "r"(v.lo.y), "r"(v.lo.z), "r"(v.lo.w), "r"(v.hi.x), "r"(v.hi.y),
                  "r"(v.hi.z), "r"(v.hi.w)
                  : "memory");

@@ -7,20 +7,18 @@
 
 namespace moe {
 
-// Layout workspace: [header | expert_count (E) | splits_acc (R x R) |
-// tile_base (E x n_tiles) | tile_tpr (R x n_tiles) | in_rank (A = T*K,
-// uint16)], the parts after the accumulators 256-byte aligned.  Tiles are
-// runs of at most TT consecutive tokens that never straddle two source
-// ranks' token blocks, so per-rank sums are sums over whole tiles.
-// tile_base[e][j] first holds the number of expert-e assignments in tile j,
-// then (after the scan) the number in all earlier tiles: the stable base of
-// tile j inside expert e's group.  in_rank[f] is the number of earlier
-// assignments of f's expert inside f's tile, so
+// Layout workspace: [header | expert_count (E) | tile_base (E x n_tiles) |
+// tile_tpr (R x n_tiles) | in_rank (A = T*K, uint16)], the parts after the
+// header 256-byte aligned.  Tiles are runs of at most TT consecutive tokens
+// that never straddle two source ranks' token blocks, so per-rank sums are
+// sums over whole tiles.  tile_base[e][j] first holds the number of expert-e
+// assignments in tile j, then (after the row scan) the number in all earlier
+// tiles: the stable base of tile j inside expert e's group.  in_rank[f] is the
+// number of earlier assignments of f's expert inside f's tile, so
 //     row(f) = expert_offsets[e] + tile_base[e][tile(t)] + in_rank[f].
-// The bytes from the header's arrival counter to the end of splits_acc are
-// zeroed before every layout launch (one memset): the cooperative layout
-// accumulates per-expert totals and per-(source, destination) splits there
-// with atomics while it ranks its tiles.
+// expert_count[e] is e's total.  Every word the layout reads is written
+// earlier in the same call (the header's arrival counter by the tile kernel,
+// before the row kernel counts on it), so a workspace needs no initialisation.
 struct LayoutHeader {
     int64_t off_tile_base;     // byte offsets of the parts (so a reader needs no R)
     int64_t off_tile_tpr;
@@ -31,7 +29,7 @@ struct LayoutHeader {
     int32_t TT;        // tokens per tile
     int32_t tpb;       // tiles per source block
     int32_t n_tiles;   // R * tpb
-    uint32_t done;     // arrival counter of the layout kernel (zeroed before each launch)
+    uint32_t done;     // arrival counter of the row kernel (zeroed by the tile kernel)
     int32_t pad[7];
 };
 static_assert(sizeof(LayoutHeader) == 96, "header layout");
@@ -74,18 +72,22 @@ inline Geometry layout_geometry(int T, int K, int R) {
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// The claim the direct expert-parallel dispatch records for a row of a
+// receive buffer: the sending rank (< 64) and its flat index f = t*K + k
+// (< 2^25) in one non-negative int32; -1 marks a row nobody holds.
+constexpr int kClaimShift = 25;
+__host__ __device__ inline int32_t claim_code(int rank, int64_t f) {
+    return (int32_t)(((uint32_t)rank << kClaimShift) | (uint32_t)f);
+}
+
 struct WsLayout {
-    size_t zero_begin, expert_count, splits_acc, zero_end;
-    size_t tile_base, tile_tpr, in_rank, total;
+    size_t expert_count, tile_base, tile_tpr, in_rank, total;
 };
 
 inline WsLayout workspace_layout(int E, int R, int n_tiles, int64_t A) {
     WsLayout w;
-    w.zero_begin = offsetof(LayoutHeader, done);
     w.expert_count = align256(sizeof(LayoutHeader));
-    w.splits_acc = w.expert_count + sizeof(int32_t) * (size_t)E;
-    w.zero_end = w.splits_acc + sizeof(int32_t) * (size_t)R * (size_t)R;
-    w.tile_base = align256(w.zero_end);
+    w.tile_base = align256(w.expert_count + sizeof(int32_t) * (size_t)E);
     w.tile_tpr = w.tile_base + align256(sizeof(int32_t) * (size_t)E * (size_t)n_tiles);
     w.in_rank = w.tile_tpr + align256(sizeof(int32_t) * (size_t)n_tiles * (size_t)R);
     w.total = w.in_rank + align256(sizeof(uint16_t) * (size_t)A);
@@ -99,16 +101,6 @@ cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, i
                           int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
                           int32_t* expert_offsets, void* workspace, int32_t* status,
                           cudaStream_t stream);
-
-// launch_layout with the grid barrier's target raised by bar_extra arrivals
-// and its wait bounded by bar_limit_ns; require_coop refuses shapes that
-// would run the non-cooperative path (cudaErrorNotSupported).
-cudaError_t launch_layout_ex(const int64_t* topk_idx, int T, int K, int E, int R, int align,
-                             int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
-                             int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
-                             int32_t* expert_offsets, void* workspace, int32_t* status,
-                             cudaStream_t stream, unsigned bar_extra, uint64_t bar_limit_ns,
-                             int require_coop);
 
 cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
                            const int32_t* expert_offsets, const void* workspace, int zero_pad,
@@ -150,24 +142,27 @@ cudaError_t launch_scatter_flat_index(const int32_t* row_flat, int64_t N, int T,
 cudaError_t launch_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int K,
                                     int E, int R, int H, const int32_t* dest_base,
                                     const void* workspace, uint16_t* const* dest_rows,
-                                    int64_t dest_cap, int rank, const int32_t* own_offsets,
-                                    const int32_t* own_counts, int zero_pad, int32_t* flat_to_row,
-                                    int32_t* status, cudaStream_t stream);
+                                    int32_t* const* dest_claims, int64_t dest_cap, int rank,
+                                    const int32_t* own_offsets, const int32_t* own_counts,
+                                    int zero_pad, int32_t* flat_to_row, int32_t* status,
+                                    cudaStream_t stream);
 
-cudaError_t launch_combine_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
-                                      const int32_t* flat_to_row, const int64_t* topk_idx, int E,
-                                      const void* weights, int weight_dtype, int T, int K, int H,
-                                      uint16_t* out, int32_t* status, cudaStream_t stream);
+cudaError_t launch_combine_from_ranks(const uint16_t* const* rows, const int32_t* const* claims,
+                                      int R, int rank, int64_t N_cap, const int32_t* flat_to_row,
+                                      const int64_t* topk_idx, int E, const void* weights,
+                                      int weight_dtype, int T, int K, int H, uint16_t* out,
+                                      int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
                               int32_t* dest_base, int32_t* own_offsets, int32_t* own_counts,
                               int32_t* max_rows, int32_t* status, cudaStream_t stream);
 
-cudaError_t launch_combine_slots_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
-                                            const int32_t* flat_to_row, const int64_t* topk_idx,
-                                            int E, const void* weights, int weight_dtype, int T,
-                                            int K, int H, uint16_t* out, int32_t* status,
-                                            cudaStream_t stream);
+cudaError_t launch_combine_slots_from_ranks(const uint16_t* const* rows,
+                                            const int32_t* const* claims, int R, int rank,
+                                            int64_t N_cap, const int32_t* flat_to_row,
+                                            const int64_t* topk_idx, int E, const void* weights,
+                                            int weight_dtype, int T, int K, int H, uint16_t* out,
+                                            int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_segment_labels(const int32_t* counts, int n, int modulo, int64_t rows,
                                   int64_t* labels, int32_t* status, cudaStream_t stream);

@@ -58,10 +58,9 @@ extern "C" int moe_dispatch_layout_noalloc(const int64_t* topk_idx, int T, int K
     void* ws = nullptr;
     const int rc = scratch_on_current_device(&ws);
     if (rc != MOE_OK) return rc;
-    // What must start at zero (the layout kernel's arrival counter and its
-    // per-expert / per-rank accumulators) is cleared by the layout itself
-    // with one memset on `stream` before its kernel, and the kernel writes
-    // every other word it later reads, so the scratch left by an earlier call
+    // What must start at zero (the row kernel's arrival counter) is zeroed
+    // by the layout's first kernel, and its kernels write every other word
+    // they read before reading it, so the scratch left by an earlier call
     // needs no clearing here.
     return moe_dispatch_layout(topk_idx, T, K, E, R, align, tokens_per_expert, counts, splits,
                                tokens_per_rank, is_token_in_rank, expert_offsets, ws, status,

@@ -31,9 +31,9 @@ __global__ void __launch_bounds__(kBlock, 4)
 permute_to_ranks_kernel(const uint4* __restrict__ x, int n16, const int64_t* __restrict__ topk,
                         int T, int K, int E, int El, int R, const int32_t* __restrict__ dest_base,
                         const char* __restrict__ ws, uint4* const* __restrict__ dest,
-                        int64_t dest_cap, int my_rank, const int32_t* __restrict__ own_off,
-                        const int32_t* __restrict__ own_cnt, int zero_pad,
-                        int32_t* __restrict__ f2r, int32_t* __restrict__ status) {
+                        int32_t* const* __restrict__ claims, int64_t dest_cap, int my_rank,
+                        const int32_t* __restrict__ own_off, const int32_t* __restrict__ own_cnt,
+                        int zero_pad, int32_t* __restrict__ f2r, int32_t* __restrict__ status) {
     __shared__ int padstart[MOE_MAX_E + 1];
     __shared__ int scratch[kWarps + 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -55,13 +55,13 @@ permute_to_ranks_kernel(const uint4* __restrict__ x, int n16, const int64_t* __r
         padstart[el] = p > 0 ? p : 0;
     }
     __syncthreads();
-    const int P = zero_pad ? block_exclusive_scan<MOE_MAX_E / kBlock>(padstart, El, scratch) : 0;
+    const int P = block_exclusive_scan<MOE_MAX_E / kBlock>(padstart, El, scratch);
     if (tid == 0) padstart[El] = P;
     __syncthreads();
 
     const int pieces = (n16 + 32 * U - 1) / (32 * U);
     const int64_t tok_items = (int64_t)T * pieces;
-    const int64_t n_items = tok_items + (int64_t)P * pieces;
+    const int64_t n_items = tok_items + (zero_pad ? (int64_t)P * pieces : 0);
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     int bad = 0;
 
@@ -92,7 +92,10 @@ permute_to_ranks_kernel(const uint4* __restrict__ x, int n16, const int64_t* __r
                 } else if (p == 0) {
                     bad |= MOE_ST_EXPERT_OOR;
                 }
-                if (p == 0) f2r[f] = myrow;
+                if (p == 0) {
+                    f2r[f] = myrow;
+                    if (claims && myrow >= 0) claims[myrank][myrow] = claim_code(my_rank, f);
+                }
             }
             for (int k = 0; k < K; ++k) {
                 const int r = __shfl_sync(kFull, myrow, k);
@@ -117,6 +120,20 @@ permute_to_ranks_kernel(const uint4* __restrict__ x, int n16, const int64_t* __r
                 if (v0 + 32 * u < n16) st_vec(dst + v0 + 32 * u, zero);
         }
     }
+    // Claims of this rank's own buffer that no sender writes this call (its
+    // pad rows and the rows past its padded total) are cleared, so a stale
+    // row never passes the restore's check.
+    if (claims) {
+        int32_t* mine = claims[my_rank];
+        const int64_t gstride = (int64_t)gridDim.x * kBlock;
+        const int64_t g0 = (int64_t)blockIdx.x * kBlock + tid;
+        for (int64_t q = g0; q < P; q += gstride) {
+            const int el = upper_index(padstart, El + 1, (int)q);
+            const int64_t row = (int64_t)own_off[el] + own_cnt[el] + (q - padstart[el]);
+            if (row >= 0 && row < dest_cap) mine[row] = -1;
+        }
+        for (int64_t row = (int64_t)own_off[El] + g0; row < dest_cap; row += gstride) mine[row] = -1;
+    }
     warp_status_or(status, bad);
 }
 
@@ -126,10 +143,12 @@ permute_to_ranks_kernel(const uint4* __restrict__ x, int n16, const int64_t* __r
 // single-device restore of the same rows.
 template <int U>
 __global__ void __launch_bounds__(kBlock)
-combine_from_ranks_kernel(const uint4* const* __restrict__ rows, int R, int64_t N_cap,
-                          const int32_t* __restrict__ f2r, const int64_t* __restrict__ topk,
-                          int E, int El, const void* __restrict__ w, int wdtype, int T, int K,
-                          int n16, uint4* __restrict__ out, int32_t* __restrict__ status) {
+combine_from_ranks_kernel(const uint4* const* __restrict__ rows,
+                          const int32_t* const* __restrict__ claims, int my_rank, int R,
+                          int64_t N_cap, const int32_t* __restrict__ f2r,
+                          const int64_t* __restrict__ topk, int E, int El,
+                          const void* __restrict__ w, int wdtype, int T, int K, int n16,
+                          uint4* __restrict__ out, int32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     pdl_wait();
     pdl_trigger();
@@ -148,6 +167,7 @@ combine_from_ranks_kernel(const uint4* const* __restrict__ rows, int R, int64_t 
                 myrow = r;
                 myrank = (int)(e / El);
                 myw = load_weight(w, wdtype, f);
+                if (claims && claims[myrank][r] != claim_code(my_rank, f)) bad |= MOE_ST_COVERAGE;
             }
         }
         uint4* dst = out + (size_t)t * n16;
@@ -252,9 +272,10 @@ cudaError_t launch_rank_bases(const int32_t* all_counts, int R, int E, int rank,
 cudaError_t launch_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int K,
                                     int E, int R, int H, const int32_t* dest_base,
                                     const void* workspace, uint16_t* const* dest_rows,
-                                    int64_t dest_cap, int rank, const int32_t* own_offsets,
-                                    const int32_t* own_counts, int zero_pad, int32_t* flat_to_row,
-                                    int32_t* status, cudaStream_t stream) {
+                                    int32_t* const* dest_claims, int64_t dest_cap, int rank,
+                                    const int32_t* own_offsets, const int32_t* own_counts,
+                                    int zero_pad, int32_t* flat_to_row, int32_t* status,
+                                    cudaStream_t stream) {
     constexpr int U = 8;
     const int n16 = H / 8;
     const int El = E / R;
@@ -267,27 +288,29 @@ cudaError_t launch_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, 
     return launch_pdl(permute_to_ranks_kernel<U>, dim3((int)grid), dim3(kBlock), 0, stream,
                       reinterpret_cast<const uint4*>(x), n16, topk_idx, T, K, E, El, R, dest_base,
                       static_cast<const char*>(workspace),
-                      reinterpret_cast<uint4* const*>(dest_rows), dest_cap, rank, own_offsets,
-                      own_counts, zero_pad, flat_to_row, status);
+                      reinterpret_cast<uint4* const*>(dest_rows), dest_claims, dest_cap, rank,
+                      own_offsets, own_counts, zero_pad, flat_to_row, status);
 }
 
-cudaError_t launch_combine_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
-                                      const int32_t* flat_to_row, const int64_t* topk_idx, int E,
-                                      const void* weights, int weight_dtype, int T, int K, int H,
-                                      uint16_t* out, int32_t* status, cudaStream_t stream) {
+cudaError_t launch_combine_from_ranks(const uint16_t* const* rows, const int32_t* const* claims,
+                                      int R, int rank, int64_t N_cap, const int32_t* flat_to_row,
+                                      const int64_t* topk_idx, int E, const void* weights,
+                                      int weight_dtype, int T, int K, int H, uint16_t* out,
+                                      int32_t* status, cudaStream_t stream) {
     // K <= 8: the slot-major restore of combine.cu (contiguous row chunks,
     // several in flight per warp) reading each slot from its rank's buffer.
     if (K <= 8)
-        return launch_combine_slots_from_ranks(rows, R, N_cap, flat_to_row, topk_idx, E, weights,
-                                               weight_dtype, T, K, H, out, status, stream);
+        return launch_combine_slots_from_ranks(rows, claims, R, rank, N_cap, flat_to_row, topk_idx,
+                                               E, weights, weight_dtype, T, K, H, out, status,
+                                               stream);
     constexpr int U = 2;
     const int sms = sm_count_current_device();
     int64_t grid = ((int64_t)T + kWarps - 1) / kWarps;
     if (grid > (int64_t)sms * 8) grid = (int64_t)sms * 8;
     if (grid < 1) grid = 1;
     return launch_pdl(combine_from_ranks_kernel<U>, dim3((int)grid), dim3(kBlock), 0, stream,
-                      reinterpret_cast<const uint4* const*>(rows), R, N_cap, flat_to_row,
-                      topk_idx, E, E / R, weights, weight_dtype, T, K, H / 8,
+                      reinterpret_cast<const uint4* const*>(rows), claims, rank, R, N_cap,
+                      flat_to_row, topk_idx, E, E / R, weights, weight_dtype, T, K, H / 8,
                       reinterpret_cast<uint4*>(out), status);
 }
 

@@ -247,23 +247,29 @@ class DirectHandle:
 
 def ep_dispatch_direct(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int,
                        dest_table: torch.Tensor, dest_cap: int, align: int = 1, group=None,
-                       status: torch.Tensor | None = None) -> DirectHandle:
+                       status: torch.Tensor | None = None,
+                       claims_table: torch.Tensor | None = None) -> DirectHandle:
     """Dispatch into the receive buffers listed in dest_table (one address
     per rank of `group`, each buffer [dest_cap, H] bf16).  One all-gather of
-    the per-expert counts; the rows go out inside the permute."""
+    the per-expert counts; the rows go out inside the permute.  With
+    claims_table (one int32 [dest_cap] array address per rank, mapped like
+    the buffers) the rows' claims are recorded for the combine's check."""
     rank = dist.get_rank(group)
     st = status if status is not None else api.new_status(x.device)
     lay = api.dispatch_layout(topk_idx, num_experts, 1, 1, status=st)
     _, dest_base, own_off, own_cnt = direct_plan(lay.tokens_per_expert, group, align, st)
     f2r = api.permute_to_ranks(x, topk_idx, lay, dest_base, dest_table, dest_cap, rank, own_off,
-                               own_cnt, status=st)
+                               own_cnt, claims_table=claims_table, status=st)
     return DirectHandle(lay, f2r, own_off, own_cnt, st)
 
 
 def ep_combine_direct(rows_table: torch.Tensor, N_cap: int, H: int, handle: DirectHandle,
-                      topk_idx: torch.Tensor, weights: torch.Tensor) -> torch.Tensor:
+                      topk_idx: torch.Tensor, weights: torch.Tensor,
+                      claims_table: torch.Tensor | None = None, group=None) -> torch.Tensor:
     """fused_weighted_restore of this rank's tokens, each slot read from the
     expert-output buffer of its expert's rank (rows_table: one address per
-    rank)."""
+    rank); with the dispatch's claims_table, the coverage check."""
     return api.combine_from_ranks(rows_table, N_cap, H, handle.flat_to_row, topk_idx,
-                                  handle.layout.E, weights, status=handle.status)
+                                  handle.layout.E, weights, claims_table=claims_table,
+                                  rank=dist.get_rank(group) if claims_table is not None else 0,
+                                  status=handle.status)

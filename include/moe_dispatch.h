@@ -47,12 +47,12 @@
  *  - Every data pointer is caller-owned DEVICE memory of the current device.
  *    The library allocates nothing and never synchronises with the host;
  *    every call only enqueues work on `stream` (a cudaStream_t; NULL is the
- *    legacy default stream) and returns: kernels, plus for the layout one
- *    memset of its workspace counter and accumulators (4 + 4E + 4R*R bytes).
- *    Results are defined once the stream reaches them.  The streaming
- *    kernels use programmatic dependent launch: each waits for the kernel
- *    before it on the stream to complete before its first memory access, so
- *    the order the caller sees is plain stream order.  The only state kept
+ *    legacy default stream) and returns: kernels, plus for the folded
+ *    restore's scatter one memset of its output.
+ *    Results are defined once the stream reaches them.  The kernels use
+ *    programmatic dependent launch: each waits for the kernel before it on
+ *    the stream to complete before its first memory access, so the order the
+ *    caller sees is plain stream order.  The only state kept
  *    between calls is per-device caches of launch attributes (SM count,
  *    cooperative-launch support, the layout's shared-memory opt-in).
  *  - Notation: T tokens, H hidden size (bf16 elements per row), E experts,
@@ -99,7 +99,7 @@ extern "C" {
 #define MOE_ST_ROW_OOR 4          /* a flat_to_row entry outside [0, N_cap)     */
 #define MOE_ST_COVERAGE 8         /* row maps do not cover each (token, slot) once */
 #define MOE_ST_LAYOUT_MISMATCH 16 /* workspace was built for another (T, K, E)  */
-#define MOE_ST_TIMEOUT 32         /* a bounded grid barrier gave up (outputs
+#define MOE_ST_TIMEOUT 32         /* a bounded wait in a kernel gave up (outputs
                                      undefined; the kernel returned)         */
 
 /* Routing-weight ("router") dtypes. */
@@ -147,13 +147,11 @@ int64_t moe_worst_case_rows(int T, int K, int E, int align);
  *                                     takes no rows)
  *      workspace                      moe_layout_workspace_bytes(T,K,E,R)
  *                                     bytes, 16-byte aligned
- * Launch: a memset of the workspace's counter and accumulators, then one
- * kernel of about one 1024-thread CTA per SM, cooperative (its tile ranking
- * and its scans are separated by one grid barrier) when all its CTAs fit on
- * the GPU at once; a barrier that does not complete within 2 s gives up and
- * sets MOE_ST_TIMEOUT.
- * Status: MOE_ST_EXPERT_OOR (that assignment is left out of every count),
- *         MOE_ST_TIMEOUT.
+ * Launch: two kernels, chained with programmatic dependent launch: one
+ * 1024-thread CTA per tile of tokens ranks the assignments, then one warp per
+ * row of per-tile counts scans it; the last of those CTAs writes the
+ * offsets.  No memset, no grid barrier, no cooperative launch.
+ * Status: MOE_ST_EXPERT_OOR (that assignment is left out of every count).
  * Errors: MOE_ERR_INVALID_ARG for a null pointer, sizes outside the limits,
  *         align < 1, misalignment. */
 int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int align,
@@ -161,26 +159,6 @@ int moe_dispatch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int
                         int32_t* tokens_per_rank, uint8_t* is_token_in_rank,
                         int32_t* expert_offsets, void* workspace, int32_t* status,
                         cudaStream_t stream);
-
-/* TEST ONLY -- not part of the path.  The pages have no counterpart: this
- * call exists so that a test can watch the layout's bounded grid barrier
- * give up.  It runs moe_dispatch_layout (same arguments and buffers) with the
- * barrier's target set one arrival above the number of CTAs, which no launch
- * can reach, and with the wait bounded by limit_ns nanoseconds (0 to
- * 100,000,000) instead of 2 s.  Every CTA then waits limit_ns, gives up,
- * sets MOE_ST_TIMEOUT and returns: the kernel ends after about limit_ns, the
- * context stays usable, and the outputs written after the barrier
- * (tokens_per_expert, counts, splits, tokens_per_rank, expert_offsets) are
- * left untouched; is_token_in_rank and the workspace are written before it.
- * Errors: as moe_dispatch_layout, plus MOE_ERR_INVALID_ARG for a limit out
- * of range or for sizes whose layout would not run the cooperative
- * (barrier) path on this device. */
-int moe_dispatch_layout_timeout_test(const int64_t* topk_idx, int T, int K, int E, int R,
-                                     int align, int32_t* tokens_per_expert, int32_t* counts,
-                                     int32_t* splits, int32_t* tokens_per_rank,
-                                     uint8_t* is_token_in_rank, int32_t* expert_offsets,
-                                     void* workspace, int32_t* status, int64_t limit_ns,
-                                     cudaStream_t stream);
 
 /* moe_dispatch_layout for callers that cannot allocate device memory.  The
  * pages have no counterpart of this call; it exists for callers such as a
@@ -204,9 +182,9 @@ int moe_dispatch_layout_timeout_test(const int64_t* topk_idx, int T, int K, int 
  *    (which destroys that context and the library's device array with it)
  *    this call is not supported in the same process.
  *  - Every call shares the one array, which keeps the last call's contents;
- *    the call clears what must start at zero (a memset of the layout's
- *    counter and accumulators, enqueued on `stream`) and its kernel rewrites
- *    every other word it reads, so the caller clears nothing.
+ *    the call clears what must start at zero (its first kernel zeroes the
+ *    arrival counter its second kernel counts on) and its kernels write every
+ *    other word they read before reading it, so the caller clears nothing.
  *    Calls that overlap on the GPU -- on different streams, or from threads
  *    whose streams are not ordered -- race on it and give undefined results.
  *  - The permute cannot use this scratch; a caller that also permutes uses
@@ -426,8 +404,12 @@ int moe_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
  *      in-tile ranks; checked on the device: MOE_ST_LAYOUT_MISMATCH),
  *      dest_rows: DEVICE array of R pointers to bf16 buffers [dest_cap, H]
  *      (16-byte aligned; across GPUs, peer addresses of the other ranks'
- *      buffers, written with plain stores), own_offsets [E/R + 1] and
- *      own_counts [E/R] int32: this rank's padded group starts and real rows.
+ *      buffers, written with plain stores), dest_claims: NULL, or a DEVICE
+ *      array of R pointers to int32 arrays [dest_cap] beside those buffers:
+ *      every row stored gets the claim (rank << 25) | f, and this rank's own
+ *      pad rows and rows past its padded total get -1 (needs T*K <= 2^25),
+ *      own_offsets [E/R + 1] and own_counts [E/R] int32: this rank's padded
+ *      group starts and real rows.
  * Out: the rows in the ranks' buffers; flat_to_row [T,K] int32 = row(f) in
  *      the buffer of its expert's rank (-1 if none).
  * Status: MOE_ST_EXPERT_OOR, MOE_ST_CAPACITY (a row at or past dest_cap is
@@ -438,9 +420,10 @@ int moe_rank_bases(const int32_t* all_counts, int R, int E, int rank, int align,
  *         GPUs: a barrier between this call and the experts). */
 int moe_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int R,
                          int H, const int32_t* dest_base, const void* workspace,
-                         uint16_t* const* dest_rows, int64_t dest_cap, int rank,
-                         const int32_t* own_offsets, const int32_t* own_counts, int zero_pad,
-                         int32_t* flat_to_row, int32_t* status, cudaStream_t stream);
+                         uint16_t* const* dest_rows, int32_t* const* dest_claims,
+                         int64_t dest_cap, int rank, const int32_t* own_offsets,
+                         const int32_t* own_counts, int zero_pad, int32_t* flat_to_row,
+                         int32_t* status, cudaStream_t stream);
 
 /* Combine straight out of the ranks' expert-output buffers: the
  * fused_weighted_restore of [DS-8847] for this rank's T tokens, slot (t, k)
@@ -453,20 +436,23 @@ int moe_permute_to_ranks(const uint16_t* x, const int64_t* topk_idx, int T, int 
  * bit-identical to the single-device restore of the same rows.
  * In:  rows: DEVICE array of R pointers to bf16 [N_cap, H] buffers (across
  *      GPUs, peer addresses; plain loads), flat_to_row [T,K], topk_idx [T,K],
- *      weights [T,K] fp32 or bf16.
+ *      weights [T,K] fp32 or bf16; claims: NULL, or the DEVICE array of R
+ *      claim arrays that moe_permute_to_ranks filled (peer addresses across
+ *      GPUs), with `rank` this rank's index.
  * Out: out [T,H] bf16.
  * Status: MOE_ST_ROW_OOR for a slot whose row or expert is out of range (it
- *         contributes nothing).
- * No coverage check: the ranks' buffers carry no map from a row back to the
- * (source rank, token, slot) it holds, so a stale or duplicated flat_to_row
- * inside [0, N_cap) combines the wrong rows without a status bit.  The
- * checked form is moe_combine_weighted with validate = 1 over a local
- * buffer and its row_to_flat (the all-to-all form of expert parallelism).
- * Errors: MOE_ERR_INVALID_ARG as moe_combine_weighted, plus E % R. */
-int moe_combine_from_ranks(const uint16_t* const* rows, int R, int64_t N_cap,
-                           const int32_t* flat_to_row, const int64_t* topk_idx, int E,
-                           const void* weights, int weight_dtype, int T, int K, int H,
-                           uint16_t* out, int32_t* status, cudaStream_t stream);
+ *         contributes nothing).  With claims, the coverage check of [DS-8847]
+ *         from the slot side: every slot's row must be claimed by exactly this
+ *         (rank, token, slot), else MOE_ST_COVERAGE -- a duplicated, stale or
+ *         foreign row is caught.  (Rows nobody points to are not visible to
+ *         one rank.)
+ * Errors: MOE_ERR_INVALID_ARG as moe_combine_weighted, plus E % R, and with
+ *         claims rank outside [0, R) or T*K > 2^25. */
+int moe_combine_from_ranks(const uint16_t* const* rows, const int32_t* const* claims, int R,
+                           int rank, int64_t N_cap, const int32_t* flat_to_row,
+                           const int64_t* topk_idx, int E, const void* weights, int weight_dtype,
+                           int T, int K, int H, uint16_t* out, int32_t* status,
+                           cudaStream_t stream);
 
 /* Backward of fused_weighted_restore ([DS-8847] Tests: row and score
  * gradients; Benchmark: score gradient in FP32; [DeepEP-272]: the backward

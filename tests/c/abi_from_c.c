@@ -52,7 +52,7 @@ int main(void) {
                                s) == MOE_ERR_INVALID_ARG);                      /* null w */
     CHECK(moe_segment_labels((const int32_t*)A, 0, 8, 10, (int64_t*)A, (int32_t*)A,
                              s) == MOE_ERR_INVALID_ARG);                        /* n = 0 */
-    CHECK(moe_combine_from_ranks((const uint16_t* const*)A, 3, 256, (const int32_t*)A,
+    CHECK(moe_combine_from_ranks((const uint16_t* const*)A, NULL, 3, 0, 256, (const int32_t*)A,
                                  (const int64_t*)A, 8, A, MOE_DTYPE_F32, 64, 2, 64,
                                  (uint16_t*)A, (int32_t*)A, s) == MOE_ERR_INVALID_ARG);
     CHECK(moe_dispatch_layout_noalloc((const int64_t*)A, 1 << 20, 32, 1024, 1, 1, (int32_t*)A,

@@ -142,24 +142,29 @@ def test_segment_labels_host_checks(L, kw):
 
 @pytest.mark.parametrize("kw", [dict(R=0), dict(R=3), dict(rank=4), dict(rank=-1), dict(H=60),
                                 dict(table=0), dict(table=A16 + 4), dict(base=0),
-                                dict(ws=A16 + 8), dict(cap=-1), dict(own=0)])
+                                dict(ws=A16 + 8), dict(cap=-1), dict(own=0),
+                                dict(claims=A16 + 4), dict(claims=A16, T=1 << 22, K=16)])
 def test_permute_to_ranks_host_checks(L, kw):
-    a = dict(x=A16, topk=A16, T=64, K=2, E=8, R=4, H=64, base=A16, ws=A16, table=A16, cap=256,
-             rank=0, own=A16, f2r=A16)
+    a = dict(x=A16, topk=A16, T=64, K=2, E=8, R=4, H=64, base=A16, ws=A16, table=A16, claims=None,
+             cap=256, rank=0, own=A16, f2r=A16)
     a.update(kw)
     rc = L.moe_permute_to_ranks(a["x"], a["topk"], a["T"], a["K"], a["E"], a["R"], a["H"],
-                                a["base"], a["ws"], a["table"], a["cap"], a["rank"], a["own"],
-                                a["own"], 1, a["f2r"], A16, None)
+                                a["base"], a["ws"], a["table"], a["claims"], a["cap"], a["rank"],
+                                a["own"], a["own"], 1, a["f2r"], A16, None)
     assert rc == -1
 
 
 @pytest.mark.parametrize("kw", [dict(R=3), dict(R=65), dict(rows=0), dict(rows=A16 + 4),
-                                dict(wd=2), dict(out=A16 + 8), dict(topk=0), dict(H=12)])
+                                dict(wd=2), dict(out=A16 + 8), dict(topk=0), dict(H=12),
+                                dict(claims=A16, rank=4), dict(claims=A16, rank=-1),
+                                dict(claims=A16 + 4), dict(claims=A16, T=1 << 22, K=16)])
 def test_combine_from_ranks_host_checks(L, kw):
-    a = dict(rows=A16, R=4, N=256, f2r=A16, topk=A16, E=8, w=A16, wd=0, T=64, K=2, H=64, out=A16)
+    a = dict(rows=A16, claims=None, R=4, rank=0, N=256, f2r=A16, topk=A16, E=8, w=A16, wd=0, T=64,
+             K=2, H=64, out=A16)
     a.update(kw)
-    rc = L.moe_combine_from_ranks(a["rows"], a["R"], a["N"], a["f2r"], a["topk"], a["E"], a["w"],
-                                  a["wd"], a["T"], a["K"], a["H"], a["out"], A16, None)
+    rc = L.moe_combine_from_ranks(a["rows"], a["claims"], a["R"], a["rank"], a["N"], a["f2r"],
+                                  a["topk"], a["E"], a["w"], a["wd"], a["T"], a["K"], a["H"],
+                                  a["out"], A16, None)
     assert rc == -1
 
 

@@ -164,6 +164,7 @@ def _run_emulated(inp, R, E, align):
     (4, 32, 4, 512, 256, 8, 0.0),
     (8, 64, 8, 256, 136, 16, 3.0),
     (2, 8, 2, 300, 64, 1, 0.0),
+    (2, 16, 10, 128, 64, 4, 0.0),       # K = 10: the any-K restore kernel
 ])
 def test_ep_direct_emulated(R, E, K, Tb, H, align, skew):
     T = R * Tb
@@ -185,7 +186,10 @@ def _run_direct(inp, R, E, align):
     """Every rank stores its rows straight into the R receive buffers (a
     table of addresses: separate buffers on this one GPU, peer addresses
     across GPUs) and gathers the expert outputs straight from them; the row
-    bases come from the library's moe_rank_bases on the gathered counts."""
+    bases come from the library's moe_rank_bases on the gathered counts.
+    The rows' claims (which rank's token and slot each row holds) equal the
+    oracle's, and the restore's coverage check from them catches planted
+    duplicates and unclaimed rows."""
     from combine_moe_dispatch_03_b200 import api, ep
     dev = torch.device("cuda:0")
     T, K = inp["topk_idx"].shape
@@ -205,12 +209,26 @@ def _run_direct(inp, R, E, align):
     recv = [torch.full((cap, H), 0x3F80, dtype=torch.int16, device=dev).view(torch.bfloat16)
             for _ in range(R)]
     table = torch.tensor([b.data_ptr() for b in recv], dtype=torch.int64, device=dev)
+    claims = [torch.full((cap,), 12345, dtype=torch.int32, device=dev) for _ in range(R)]
+    ctable = torch.tensor([c.data_ptr() for c in claims], dtype=torch.int64, device=dev)
     f2rs, owns = [], []
     for s in range(R):
         dest_base, own_off, own_cnt = ep.rank_bases(all_counts, s, align, status=st)
         owns.append((own_off, own_cnt))
         f2rs.append(api.permute_to_ranks(blk(x, s), blk(tk, s), lays[s], dest_base, table, cap, s,
-                                         own_off, own_cnt, status=st))
+                                         own_off, own_cnt, claims_table=ctable, status=st))
+    # Every row's claim, from the oracle's single-device rows: a real row of
+    # owner r holds (source rank, that rank's flat index); pads and the rows
+    # past the padded total hold -1.
+    topk_np = inp["topk_idx"].numpy()
+    o_r2f = orc.permute(np.zeros((T, 8), np.uint16), topk_np, E, off, int(off[-1]))["row_to_flat"]
+    for r in range(R):
+        lo, hi = int(off[r * El]), int(off[(r + 1) * El])
+        g = o_r2f[lo:hi].astype(np.int64)
+        t, k = g // K, g % K
+        want = np.where(g >= 0, ((t // Tb) << 25) | ((t % Tb) * K + k), -1)
+        want = np.concatenate([want, np.full(cap - (hi - lo), -1)]).astype(np.int32)
+        np.testing.assert_array_equal(claims[r].cpu().numpy(), want, err_msg=f"claims of rank {r}")
     ys = []
     for r in range(R):
         own_off, own_cnt = owns[r]
@@ -225,10 +243,39 @@ def _run_direct(inp, R, E, align):
     ytab = torch.tensor([y.data_ptr() for y in ys], dtype=torch.int64, device=dev)
     outs = []
     for s in range(R):
-        out_s = api.combine_from_ranks(ytab, cap, H, f2rs[s], blk(tk, s), E, blk(w, s), status=st)
+        out_s = api.combine_from_ranks(ytab, cap, H, f2rs[s], blk(tk, s), E, blk(w, s),
+                                       claims_table=ctable, rank=s, status=st)
         _check_out(out_s, o, s, Tb, f"rank {s} output")
         outs.append(out_s)
     api.check_status(st)
+    # Planted faults, caught by the claims: a slot given another slot's row
+    # of the same owner (a duplicate), a slot given a row past its owner's
+    # padded total (claimed by nobody), and rank 1's slots checked as rank 0's.
+    owner = (topk_np[:Tb] // El).reshape(-1)
+    f1, f2 = next((a, b) for a in range(owner.size) for b in range(a + 1, owner.size)
+                  if owner[a] == owner[b])
+    own_total = {r: int(off[(r + 1) * El] - off[r * El]) for r in range(R)}
+    faults = []
+    dup = f2rs[0].clone().view(-1)
+    dup[f1] = dup[f2]
+    faults.append(dup.view(Tb, K))
+    if own_total[int(owner[0])] < cap:
+        past = f2rs[0].clone().view(-1)
+        past[0] = cap - 1
+        faults.append(past.view(Tb, K))
+    for bad in faults:
+        st_bad = api.new_status(dev)
+        api.combine_from_ranks(ytab, cap, H, bad, blk(tk, 0), E, blk(w, 0), claims_table=ctable,
+                               rank=0, status=st_bad)
+        assert int(st_bad.item()) & 8, "a duplicated or unclaimed row must set MOE_ST_COVERAGE"
+    st_free = api.new_status(dev)                     # without claims: not checked
+    api.combine_from_ranks(ytab, cap, H, faults[0], blk(tk, 0), E, blk(w, 0), status=st_free)
+    assert int(st_free.item()) == 0
+    if R > 1:
+        st_rank = api.new_status(dev)
+        api.combine_from_ranks(ytab, cap, H, f2rs[1], blk(tk, 1), E, blk(w, 1),
+                               claims_table=ctable, rank=0, status=st_rank)
+        assert int(st_rank.item()) & 8
     lay = api.dispatch_layout(tk, E, R, align, status=st)
     xp, _, f2r = api.permute(x, tk, lay, status=st)
     out_ref = api.combine_weighted(api.expert_scale(xp, lay, sc, status=st), f2r, w, status=st)

@@ -253,57 +253,3 @@ def test_host_checks_launch_nothing(case):
     torch.cuda.synchronize()
     assert st.item() == 0
     assert not xp.view(torch.int16).any() and not r2f.any() and not f2r.any()
-
-
-@pytest.mark.parametrize("T,K,E,R,align", [(4096, 8, 128, 8, 16), (64, 2, 8, 2, 8)])
-def test_layout_grid_barrier_gives_up(T, K, E, R, align):
-    """The cooperative layout's grid barrier is a bounded wait.  The test-only
-    entry point raises the barrier's target one arrival above the number of
-    CTAs (so it can never complete) and bounds the wait at 1 ms: the call
-    must return within a fraction of a second with MOE_ST_TIMEOUT set, leave
-    every output written after the barrier untouched (canaries), and leave
-    the context usable -- the ordinary layout on the same buffers right after
-    matches the oracle."""
-    import time
-
-    import oracle as orc
-    from combine_moe_dispatch_03_b200 import _lib
-    api = _api()
-    dev = torch.device("cuda:0")
-    inp = custom_inputs(T, 16, E, K, seed=23)
-    topk = inp["topk_idx"].to(dev)
-    lay = api.alloc_layout(T, K, E, R, align, dev)
-    for t in (lay.tokens_per_expert, lay.counts, lay.splits, lay.tokens_per_rank,
-              lay.expert_offsets):
-        t.fill_(-7)
-    st = api.new_status(dev)
-    P = lambda t: t.data_ptr()
-    torch.cuda.synchronize(dev)
-    t0 = time.perf_counter()
-    rc = _lib.lib().moe_dispatch_layout_timeout_test(
-        P(topk), T, K, E, R, align, P(lay.tokens_per_expert), P(lay.counts), P(lay.splits),
-        P(lay.tokens_per_rank), P(lay.is_token_in_rank), P(lay.expert_offsets), P(lay.workspace),
-        P(st), 1_000_000, torch.cuda.current_stream(dev).cuda_stream)
-    assert rc == _lib.MOE_OK
-    torch.cuda.synchronize(dev)
-    elapsed = time.perf_counter() - t0
-    assert elapsed < 0.5, elapsed
-    assert int(st.item()) == _lib.ST_TIMEOUT
-    for t in (lay.tokens_per_expert, lay.counts, lay.splits, lay.tokens_per_rank,
-              lay.expert_offsets):
-        assert bool((t == -7).all())
-    # limits the entry point refuses
-    bad = _lib.lib().moe_dispatch_layout_timeout_test(
-        P(topk), T, K, E, R, align, P(lay.tokens_per_expert), P(lay.counts), P(lay.splits),
-        P(lay.tokens_per_rank), P(lay.is_token_in_rank), P(lay.expert_offsets), P(lay.workspace),
-        P(st), 10 ** 9, torch.cuda.current_stream(dev).cuda_stream)
-    assert bad == _lib.MOE_ERR_INVALID_ARG
-    # the context and the buffers are still good
-    st2 = api.new_status(dev)
-    api.dispatch_layout(topk, E, R, align, status=st2, out=lay)
-    torch.cuda.synchronize(dev)
-    assert int(st2.item()) == 0
-    want = orc.layout(inp["topk_idx"].numpy(), E, R, align)
-    for name in ("tokens_per_expert", "counts", "splits", "tokens_per_rank", "is_token_in_rank",
-                 "expert_offsets"):
-        np.testing.assert_array_equal(getattr(lay, name).cpu().numpy(), want[name], err_msg=name)

@@ -1,6 +1,6 @@
 """(1) The whole forward + backward step captured in a CUDA graph replays
 bit-identically to eager execution (no call allocates or synchronises, so the
-chain is capturable; the layout's memset and cooperative launch included).
+chain is capturable; the layout's two kernels included).
 (2) At the four shapes of the pages' benchmark table (DeepSpeed PR "AutoEP:
 support combine_impl=fused_weighted_sum with AutoEP+AutoTP folding",
 Benchmark: hidden 6144, top-4 of 128 and top-8 of 256 experts, 8,192 and

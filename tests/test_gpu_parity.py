@@ -73,9 +73,10 @@ def test_tiny_twice_deterministic():
     (256, 16, 1024, 4, 64, 1),   # E=1024 and R=64 (maxima)
     (130, 8192, 8, 2, 2, 16),    # wide rows
     (66, 8200, 4, 2, 2, 8),      # long rows
-    (20000, 8, 64, 8, 1, 4),     # 148 tiles: the cooperative path with every SM busy
-    (40000, 8, 64, 8, 1, 4),     # 157 tiles (> 148 SMs): last-CTA path, count matrix staged
-    (9728, 8, 1024, 32, 8, 1),   # 152 tiles: last-CTA path, count matrix too big to stage
+    (20000, 8, 64, 8, 1, 4),     # 148 layout tiles, one per SM
+    (40000, 8, 64, 8, 1, 4),     # 157 tiles: more tiles than SMs
+    (9728, 8, 1024, 32, 8, 1),   # 152 tiles x 1032 rows of per-tile counts
+    (120000, 8, 16, 8, 2, 8),    # 470 tiles: rows longer than 32 x 8 tiles (several loads per lane)
 ])
 def test_edge_shapes(T, H, E, K, R, align):
     inp = custom_inputs(T, H, E, K, seed=T * 7 + K)

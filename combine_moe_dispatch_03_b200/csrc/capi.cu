@@ -353,7 +353,7 @@ const char* moe_status_bit_name(int bit) {
         case MOE_ST_ROW_OOR: return "flat_to_row entry outside [0, N_cap)";
         case MOE_ST_COVERAGE: return "row maps do not cover every (token, slot) exactly once";
         case MOE_ST_LAYOUT_MISMATCH: return "layout workspace was built for other sizes";
-        case MOE_ST_TIMEOUT: return "a bounded grid barrier timed out (kernel returned early)";
+        case MOE_ST_TIMEOUT: return "a bounded wait in a kernel timed out (kernel returned early)";
         default: return "unknown status bit";
     }
 }

@@ -50,8 +50,10 @@ def _setup(T=128, H=64, E=8, K=2, R=2, align=4, topk=None):
     return api, dev, inp
 
 
-def test_expert_out_of_range_is_flagged_and_contained():
-    T, H, E, K = 128, 64, 8, 2
+# K = 2 runs the copy-engine permute, K = 4 the register permute.
+@pytest.mark.parametrize("K", [2, 4])
+def test_expert_out_of_range_is_flagged_and_contained(K):
+    T, H, E = 128, 64, 8
     topk = torch.randint(0, E, (T, K), generator=torch.Generator().manual_seed(1))
     topk[5, 1] = -1
     topk[77, 0] = E
@@ -77,8 +79,9 @@ def test_expert_out_of_range_is_flagged_and_contained():
         api.check_status(st2)
 
 
-def test_capacity_overflow_is_flagged_and_contained():
-    T, H, E, K, align = 64, 32, 8, 2, 16
+@pytest.mark.parametrize("K", [2, 4])
+def test_capacity_overflow_is_flagged_and_contained(K):
+    T, H, E, align = 64, 32, 8, 16
     api, dev, inp = _setup(T, H, E, K)
     lay = api.dispatch_layout(inp["topk_idx"].to(dev), E, 1, align)
     n_pad = int(lay.expert_offsets[-1])
@@ -158,21 +161,22 @@ def test_row_out_of_range_is_flagged_and_skipped():
     assert torch.equal(out[2].view(torch.int16), want.view(torch.int16))
 
 
-def test_workspace_mismatch_writes_nothing():
-    api, dev, inp = _setup(64, 32, 8, 2)
+@pytest.mark.parametrize("K", [2, 4])
+def test_workspace_mismatch_writes_nothing(K):
+    api, dev, inp = _setup(64, 32, 8, K)
     lay = api.dispatch_layout(inp["topk_idx"].to(dev), 8, 2, 4)
-    inp2 = custom_inputs(32, 32, 8, 2, seed=3)
-    N = capacity_rows(32, 2, 8, 4)
+    inp2 = custom_inputs(32, 32, 8, K, seed=3)
+    N = capacity_rows(32, K, 8, 4)
     xp = torch.full((N, 32), 7, dtype=torch.int16, device=dev).view(torch.bfloat16)
     r2f = torch.full((N,), 7, dtype=torch.int32, device=dev)
-    f2r = torch.full((32, 2), 7, dtype=torch.int32, device=dev)
+    f2r = torch.full((32, K), 7, dtype=torch.int32, device=dev)
     st = api.new_status(dev)
     # Through the C ABI: the Python layer would refuse this on the host (see
     # test_python_layer_refuses_mismatched_shapes); the device check is what
     # guards a C caller.
     from combine_moe_dispatch_03_b200._lib import lib
     x2, t2 = inp2["x"].to(dev), inp2["topk_idx"].to(dev)
-    rc = lib().moe_permute(x2.data_ptr(), t2.data_ptr(), 32, 2, 8, 32,
+    rc = lib().moe_permute(x2.data_ptr(), t2.data_ptr(), 32, K, 8, 32,
                            lay.expert_offsets.data_ptr(), lay.workspace.data_ptr(), 1, N,
                            xp.data_ptr(), r2f.data_ptr(), f2r.data_ptr(), st.data_ptr(),
                            torch.cuda.current_stream().cuda_stream)

@@ -82,11 +82,11 @@ STAND_IN = ("expert_scale", "expert_scale_bwd")
 KERNELS_PER_CALL = {"layout": 2}
 
 # Step names -> the kernel function each launches at top_k = K: the permute
-# moves rows with the copy engine at K <= 2; above K = 8 the combines use
-# their any-K kernels.
+# streams rows through its shared-memory ring at K <= 2; above K = 8 the
+# combines use their any-K kernels.
 def kernel_function(name: str, K: int) -> str:
     if name == "permute":
-        return "permute_bulk_kernel" if K <= 2 else "permute_kernel"
+        return "permute_ring_kernel" if K <= 2 else "permute_kernel"
     if name in ("combine", "dispatch_backward"):
         return "combine_slots_kernel" if K <= 8 else "combine_kernel"
     if name == "combine_backward":

@@ -143,10 +143,9 @@ __device__ __forceinline__ void st_vec32(uint4* p, const Vec32& v) {
 
 // ------------------------------------------------------- bulk (TMA) copies ---
 //
-// Non-tensor bulk copies between global and shared memory done by the SM's
-// copy engine: a load completes on an mbarrier (its transaction count), a
-// store is tracked by bulk groups.  Addresses and sizes are multiples of 16
-// bytes.  No multicast form is used anywhere.
+// Non-tensor bulk loads from global into shared memory done by the SM's
+// copy engine, completing on an mbarrier (its transaction count).  Addresses
+// and sizes are multiples of 16 bytes.  No multicast form is used anywhere.
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -168,6 +167,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
                  : "memory");
 }
 
+// One arrival (no transaction bytes) of the calling thread.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 // One bounded probe of phase `parity`; true once that phase has completed.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
     uint32_t done;
@@ -187,33 +191,6 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, unsi
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_addr(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
-}
-
-__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, unsigned bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
-                 "r"(smem_addr(smem_src)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until at most N committed bulk groups still read shared memory.
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-// Wait until every committed bulk group has completed (writes performed).
-__device__ __forceinline__ void bulk_wait_all() {
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-// Orders this thread's generic-proxy shared-memory writes before later
-// copy-engine reads of them.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ------------------------------------------------------------- warp/block ---

@@ -50,7 +50,7 @@ def _setup(T=128, H=64, E=8, K=2, R=2, align=4, topk=None):
     return api, dev, inp
 
 
-# K = 2 runs the copy-engine permute, K = 4 the register permute.
+# K = 2 runs the ring permute, K = 4 the register permute.
 @pytest.mark.parametrize("K", [2, 4])
 def test_expert_out_of_range_is_flagged_and_contained(K):
     T, H, E = 128, 64, 8

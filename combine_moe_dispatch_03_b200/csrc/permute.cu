@@ -177,7 +177,7 @@ permute_kernel(const uint4* __restrict__ x, int n16, const uint32_t* __restrict_
 
 // ------------------------------------------------------ ring permute ---
 //
-// The same items, rows and maps again, for fan-out K <= 2, arranged so that
+// The same rows and maps again, for fan-out K <= 2, arranged so that
 // a small problem has nearly all of its token rows in flight at once: one
 // CTA per SM owns a contiguous range of token pieces (balanced to within one
 // piece) and a ring of S 4 KB shared-memory buffers.  Thread 0 issues the
@@ -198,7 +198,7 @@ permute_kernel(const uint4* __restrict__ x, int n16, const uint32_t* __restrict_
 // stores issued by one thread instead of the consumer warps' stores, 45 us.
 constexpr int kRingPiece = 4096;
 constexpr unsigned kRingSpinLimit = 1u << 22;
-constexpr int kRingTokens = 1024;     // tokens whose rows one CTA holds (K <= 2)
+constexpr int kRingRows = 2048;       // rows (token, slot) one CTA's row table holds
 #ifndef MOE_RING_FIRST
 #define MOE_RING_FIRST 4
 #endif
@@ -206,8 +206,8 @@ constexpr int kRingFirst = MOE_RING_FIRST;   // pieces requested before the rows
 
 template <int S>
 struct RingSmem {
-    static constexpr size_t rows = (size_t)S * kRingPiece;               // [kRingTokens * 2]
-    static constexpr size_t ints = rows + sizeof(int) * 2 * kRingTokens; // off, padstart
+    static constexpr size_t rows = (size_t)S * kRingPiece;           // [kRingRows]
+    static constexpr size_t ints = rows + sizeof(int) * kRingRows;   // off, padstart
     static size_t total(int E) { return ints + sizeof(int) * 2 * ((size_t)E + 1); }
 };
 
@@ -250,7 +250,7 @@ permute_ring_kernel(const char* __restrict__ x, int row_bytes, const int64_t* __
     // they fit the row table).
     const int64_t t_lo = i0 / pieces;
     const int64_t t_hi = n_my > 0 ? (i1 + pieces - 1) / pieces : t_lo;
-    if (K > 2 || t_hi - t_lo > kRingTokens) {
+    if ((t_hi - t_lo) * K > kRingRows) {
         if (tid == 0) atomicOr(status, MOE_ST_LAYOUT_MISMATCH);
         return;
     }
@@ -459,9 +459,11 @@ static cudaError_t launch_ring(const uint16_t* x, int row_bytes, const int64_t* 
         }
     }
     // One CTA per SM, more when a CTA's tokens would not fit its row table
-    // (a range of n pieces spans at most n / pieces + 2 tokens).
+    // (a range of n pieces spans at most n / pieces + 2 tokens; the caller
+    // keeps K <= kRingRows / 4, so a CTA holds at least 2 whole tokens).
     const int sms = sm_count_current_device();
-    int64_t grid = ((int64_t)T + (kRingTokens - 3)) / (kRingTokens - 2);
+    const int64_t per_cta = kRingRows / K - 2;
+    int64_t grid = ((int64_t)T + per_cta - 1) / per_cta;
     if (grid < sms) grid = sms;
     return launch_pdl(permute_ring_kernel<S>, dim3((int)grid), dim3(kBlock), smem, stream,
                       reinterpret_cast<const char*>(x), row_bytes, topk_idx, T, K, E,
@@ -516,11 +518,16 @@ cudaError_t launch_permute(const uint16_t* x, const int64_t* topk_idx, int T, in
     // kernel (measured on B200 against a copy-engine kernel with per-warp
     // two-stage buffers and bulk stores: Mixtral-shaped dispatch 49.5 vs
     // 51.4 us, the same at 32768 tokens 135.0 vs 138.4 us); larger fan-out:
-    // the register kernel.
+    // the register kernel (the ring at fan-out 8: Qwen3-shaped permute 113.0
+    // vs 97.4 us, DeepSeek-V3-shaped 237.5 vs 200.1 us).
 #ifndef MOE_RING_S
 #define MOE_RING_S 48
 #endif
-    if (K <= 2)
+#ifndef MOE_RING_MAXK
+#define MOE_RING_MAXK 2
+#endif
+    static_assert(MOE_RING_MAXK <= kRingRows / 4, "a CTA's row table holds two tokens");
+    if (K <= MOE_RING_MAXK)
         return launch_ring<MOE_RING_S>(x, 2 * H, topk_idx, T, K, E, expert_offsets, workspace,
                                        zero_pad, N_cap, x_perm, row_to_flat, flat_to_row, status,
                                        stream);

@@ -77,6 +77,14 @@ def test_tiny_twice_deterministic():
     (40000, 8, 64, 8, 1, 4),     # 157 tiles: more tiles than SMs
     (9728, 8, 1024, 32, 8, 1),   # 152 tiles x 1032 rows of per-tile counts
     (120000, 8, 16, 8, 2, 8),    # 470 tiles: rows longer than 32 x 8 tiles (several loads per lane)
+    # The ring permute (K <= 2): one CTA per SM, each a balanced range of
+    # 4 KB token pieces.
+    (100, 2048, 8, 2, 1, 16),    # fewer pieces than CTAs: idle CTAs
+    (777, 24, 5, 1, 1, 3),       # K = 1
+    (4000, 2056, 8, 2, 2, 16),   # 2 pieces per row, the last 16 bytes: ranges start mid-token
+    (3008, 4104, 1024, 2, 64, 1),  # E = 1024 (largest shared-memory footprint), 3 pieces per row
+    (160000, 8, 16, 2, 2, 8),    # more tokens than 148 CTAs' row tables hold: 157 CTAs
+    (160000, 8, 16, 1, 1, 8),    # the same at K = 1
 ])
 def test_edge_shapes(T, H, E, K, R, align):
     inp = custom_inputs(T, H, E, K, seed=T * 7 + K)

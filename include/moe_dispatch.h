@@ -54,8 +54,7 @@
  *    the stream to complete before its first memory access, so the order the
  *    caller sees is plain stream order.  The only state kept between calls
  *    is per-device caches of launch attributes (SM count, shared-memory
- *    opt-ins, resident CTAs per SM of the copy-engine permute) and the device
- *    array of moe_dispatch_layout_noalloc.
+ *    opt-ins) and the device array of moe_dispatch_layout_noalloc.
  *  - Notation: T tokens, H hidden size (bf16 elements per row), E experts,
  *    K = top_k, R logical ranks, El = E/R, align = group alignment,
  *    A = T*K assignments, flat index f = t*K + k (token t, slot k),

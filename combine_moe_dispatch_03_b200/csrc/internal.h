@@ -72,6 +72,14 @@ inline Geometry layout_geometry(int T, int K, int R) {
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// The ring permute (fan-out K <= 2): one CTA per SM streams a contiguous
+// range of 4 KB row pieces through shared-memory buffers filled by bulk
+// loads.  A CTA's table holds the rows of at most kRingRows (token, slot)
+// pairs; every mbarrier wait gives up after kRingSpinLimit probes.
+constexpr int kRingPiece = 4096;
+constexpr int kRingRows = 2048;
+constexpr unsigned kRingSpinLimit = 1u << 22;
+
 // The claim the direct expert-parallel dispatch records for a row of a
 // receive buffer: the sending rank (< 64) and its flat index f = t*K + k
 // (< 2^25) in one non-negative int32; -1 marks a row nobody holds.

@@ -196,9 +196,6 @@ permute_kernel(const uint4* __restrict__ x, int n16, const uint32_t* __restrict_
 // the rows need queue behind 29 MB of loads; warps wait at the CTA barrier
 // 44% of the time); 8, 4 or 2 pieces first, 21.7, 20.6 and 20.9 us; bulk
 // stores issued by one thread instead of the consumer warps' stores, 45 us.
-constexpr int kRingPiece = 4096;
-constexpr unsigned kRingSpinLimit = 1u << 22;
-constexpr int kRingRows = 2048;       // rows (token, slot) one CTA's row table holds
 #ifndef MOE_RING_FIRST
 #define MOE_RING_FIRST 4
 #endif

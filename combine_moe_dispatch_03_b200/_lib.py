@@ -61,6 +61,7 @@ SIGNATURES = {
                                     _P]),
     "moe_strerror": (ctypes.c_char_p, [_I]),
     "moe_status_bit_name": (ctypes.c_char_p, [_I]),
+    "moe_last_cuda_error": (ctypes.c_char_p, []),
     "moe_version": (ctypes.c_char_p, []),
 }
 
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
 def check_rc(rc: int, what: str) -> None:
     if rc != MOE_OK:
         msg = lib().moe_strerror(rc).decode()
+        if rc == MOE_ERR_CUDA:
+            msg += f": {lib().moe_last_cuda_error().decode()}"
         raise RuntimeError(f"{what} failed: {msg} (code {rc})")
 
 

@@ -30,6 +30,15 @@ int sm_count_current_device() {
     return n;
 }
 
+// The CUDA error behind the calling thread's last MOE_ERR_CUDA.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+int cuda_result(cudaError_t err) {
+    if (err == cudaSuccess) return MOE_OK;
+    g_last_cuda_error = err;
+    return MOE_ERR_CUDA;
+}
+
 }  // namespace moe
 
 namespace {
@@ -49,7 +58,7 @@ bool ncap_ok(int64_t N_cap, int T, int K) {
     return N_cap >= (int64_t)T * K && N_cap <= INT32_MAX;
 }
 
-int finish(cudaError_t err) { return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+int finish(cudaError_t err) { return moe::cuda_result(err); }
 
 struct NvtxRange {
     explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
@@ -356,6 +365,10 @@ const char* moe_status_bit_name(int bit) {
         case MOE_ST_TIMEOUT: return "a bounded wait in a kernel timed out (kernel returned early)";
         default: return "unknown status bit";
     }
+}
+
+const char* moe_last_cuda_error(void) {
+    return moe::g_last_cuda_error == cudaSuccess ? "none" : cudaGetErrorName(moe::g_last_cuda_error);
 }
 
 const char* moe_version(void) { return "moe_dispatch 0.1.0 (sm_100a)"; }

@@ -76,7 +76,10 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // range of 4 KB row pieces through shared-memory buffers filled by bulk
 // loads.  A CTA's table holds the rows of at most kRingRows (token, slot)
 // pairs; every mbarrier wait gives up after kRingSpinLimit probes.
-constexpr int kRingPiece = 4096;
+#ifndef MOE_RING_PIECE
+#define MOE_RING_PIECE 4096
+#endif
+constexpr int kRingPiece = MOE_RING_PIECE;
 constexpr int kRingRows = 2048;
 constexpr unsigned kRingSpinLimit = 1u << 22;
 
@@ -103,6 +106,10 @@ inline WsLayout workspace_layout(int E, int R, int n_tiles, int64_t A) {
 }
 
 int sm_count_current_device();
+
+// MOE_OK for cudaSuccess; otherwise records err for moe_last_cuda_error
+// (per host thread) and returns MOE_ERR_CUDA.
+int cuda_result(cudaError_t err);
 
 cudaError_t launch_layout(const int64_t* topk_idx, int T, int K, int E, int R, int align,
                           int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,

@@ -33,12 +33,15 @@ void* g_scratch_ptr[64] = {};
 // supported in the process (documented in the header).
 int scratch_on_current_device(void** out) {
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return moe::cuda_result(e);
+    if (dev < 0 || dev >= 64) return moe::cuda_result(cudaErrorInvalidDevice);
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
     if (g_scratch_ptr[dev] == nullptr) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess || p == nullptr)
-            return MOE_ERR_CUDA;
+        const cudaError_t e2 = cudaGetSymbolAddress(&p, g_layout_scratch);
+        if (e2 != cudaSuccess) return moe::cuda_result(e2);
+        if (p == nullptr) return moe::cuda_result(cudaErrorInvalidSymbol);
         g_scratch_ptr[dev] = p;
     }
     *out = g_scratch_ptr[dev];

@@ -482,6 +482,13 @@ int moe_combine_backward(const uint16_t* grad_out, const uint16_t* rows, int64_t
 const char* moe_strerror(int code);
 const char* moe_status_bit_name(int bit);
 
+/* The name of the CUDA error (e.g. "cudaErrorIllegalAddress") behind the
+ * calling host thread's most recent MOE_ERR_CUDA return, or "none".  Static
+ * text; a later MOE_ERR_CUDA on the same thread replaces it.  A sticky
+ * error from an earlier kernel surfaces at the next launch, so the call
+ * that reports it need not be the one whose kernel failed. */
+const char* moe_last_cuda_error(void);
+
 /* Library version string. */
 const char* moe_version(void);
 

@@ -35,6 +35,7 @@ int main(void) {
     CHECK(strstr(moe_strerror(MOE_ERR_INVALID_ARG), "invalid") != NULL);
     CHECK(strstr(moe_status_bit_name(MOE_ST_COVERAGE), "cover") != NULL);
     CHECK(strstr(moe_version(), "sm_100a") != NULL);
+    CHECK(strcmp(moe_last_cuda_error(), "none") == 0);     /* no CUDA failure on this thread */
 
     /* host checks: each call is refused before any CUDA call */
     CHECK(moe_dispatch_layout((const int64_t*)A, 64, 2, 8, 3, 4, (int32_t*)A, (int32_t*)A,

@@ -76,10 +76,7 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // range of 4 KB row pieces through shared-memory buffers filled by bulk
 // loads.  A CTA's table holds the rows of at most kRingRows (token, slot)
 // pairs; every mbarrier wait gives up after kRingSpinLimit probes.
-#ifndef MOE_RING_PIECE
-#define MOE_RING_PIECE 4096
-#endif
-constexpr int kRingPiece = MOE_RING_PIECE;
+constexpr int kRingPiece = 4096;
 constexpr int kRingRows = 2048;
 constexpr unsigned kRingSpinLimit = 1u << 22;
 

@@ -8,8 +8,8 @@ resident in HBM.
 
 One step = one pass of the path over one batch.  What is timed (``value``) is
 dispatch + combine, the steps of the metric:
-  forward-only workloads:   layout + permute | combine
-  fwd+bwd workloads:        layout + permute | combine + combine backward |
+  forward-only workloads:   dispatch (layout + permute, one call) | combine
+  fwd+bwd workloads:        dispatch | combine + combine backward |
                             dispatch backward (a unit-weight combine)
 The seeded stand-in expert (y = x * s_e, and its backward) runs between the
 timed segments -- the combine needs its output -- but outside the CUDA
@@ -32,7 +32,8 @@ skew) and Mixtral-shaped configurations, each with its tokens/s, step GB/s,
 fraction of the measured HBM peak and its dominant kernel's fraction.
 
 Other keys of the JSON line (rank 0 prints ONE line):
-  kernels      per dispatch/combine kernel: mean time of an eager launch
+  kernels      per dispatch/combine kernel (the layout and the permute as
+               separate calls): mean time of an eager launch
                (flushed L2 before it, CUDA events around it), share of the
                timed work, algorithmic bytes and GB/s, fraction of the
                measured peak, ncu DRAM traffic per launch while the kernel's
@@ -41,7 +42,7 @@ Other keys of the JSON line (rank 0 prints ONE line):
                stand-in is never a candidate): algorithmic bytes per launch /
                mean event-timed duration against the measured HBM copy
                bandwidth;
-  full_step    the whole path including the stand-in (7 launches for fwd+bwd)
+  full_step    the whole path including the stand-in (8 launches for fwd+bwd)
                captured in one graph, one flush per step;
   e2e          the full step through pinned host buffers with the
                host<->device copies inside the timed region;
@@ -78,8 +79,8 @@ METHOD = ("layout", "permute", "combine", "combine_backward", "dispatch_backward
 STAND_IN = ("expert_scale", "expert_scale_bwd")
 
 # Kernels one call of a step launches (the layout: a tile kernel and a row
-# kernel; every other call: one).
-KERNELS_PER_CALL = {"layout": 2}
+# kernel; the dispatch: those and the permute; every other call: one).
+KERNELS_PER_CALL = {"layout": 2, "dispatch": 3}
 
 # Step names -> the kernel function each launches at top_k = K: the permute
 # streams rows through its shared-memory ring at K <= 2; above K = 8 the
@@ -251,8 +252,9 @@ class Path:
             self.grad_x = torch.empty(T, H, **bf)
 
     def segments(self):
-        """(segment name, launches, timed) in step order."""
-        seg = [("dispatch", ("layout", "permute"), True),
+        """(segment name, calls, timed) in step order.  The dispatch segment
+        is one call (moe_dispatch: the layout, then the permute)."""
+        seg = [("dispatch", ("dispatch",), True),
                ("expert", ("expert_scale",), False)]
         if self.backward:
             seg += [("combine", ("combine", "combine_backward"), True),
@@ -265,12 +267,23 @@ class Path:
     def launches(self):
         return [n for _, calls, _ in self.segments() for n in calls]
 
+    def kernel_calls(self):
+        """The step's calls with the dispatch as its two separate calls (layout,
+        permute), so that each method kernel is timed on its own."""
+        out = []
+        for n in self.launches():
+            out += ["layout", "permute"] if n == "dispatch" else [n]
+        return out
+
     def method_launches(self):
-        return [n for n in self.launches() if n in METHOD]
+        return [n for n in self.kernel_calls() if n in METHOD]
 
     def call(self, name):
         api, c, st = self.api, self.cfg, self.status
-        if name == "layout":
+        if name == "dispatch":
+            api.dispatch(self.x, self.topk, c.E, c.R, c.align, capacity=self.N, status=st,
+                         layout_out=self.lay, out=(self.xp, self.r2f, self.f2r))
+        elif name == "layout":
             api.dispatch_layout(self.topk, c.E, c.R, c.align, status=st, out=self.lay)
         elif name == "permute":
             api.permute(self.x, self.topk, self.lay, capacity=self.N, status=st,
@@ -389,7 +402,7 @@ def time_kernels(path, steps, warmup, flush, dist, device):
     """Eager launches, one at a time: before each dispatch/combine launch an L2
     flush, then CUDA events around the launch alone (the stand-in launches
     run between them, untimed).  Returns {launch: [ms per step]}."""
-    names = path.launches()
+    names = path.kernel_calls()
     for _ in range(max(warmup, 0)):
         for n in names:
             if n in METHOD:

@@ -43,6 +43,8 @@ SIGNATURES = {
     "moe_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch_layout_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _L, _P, _P, _P, _P, _P]),
+    "moe_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _L, _P,
+                          _P, _P, _P, _P]),
     "moe_expert_scale": (_I, [_P, _L, _P, _P, _I, _I, _P, _P, _P, _P]),
     "moe_combine_weighted": (_I, [_P, _L, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "moe_combine_backward": (_I, [_P, _P, _L, _P, _P, _P, _I, _I, _I, _I, _P, _I, _I, _P, _P, _P,

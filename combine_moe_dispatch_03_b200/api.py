@@ -177,6 +177,45 @@ def permute(x: torch.Tensor, topk_idx: torch.Tensor, layout: Layout, capacity: i
     return x_perm, r2f, f2r
 
 
+def dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, num_ranks: int = 1,
+             align: int = 1, capacity: int | None = None, zero_pad: bool = True,
+             status: torch.Tensor | None = None, layout_out: Layout | None = None,
+             out: tuple | None = None):
+    """dispatch_layout and permute in one call (moe_dispatch).  Returns
+    (layout, x_perm, row_to_flat, flat_to_row)."""
+    _require(x, "x", torch.bfloat16, 2)
+    _require(topk_idx, "topk_idx", torch.int64, 2)
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    dev = x.device
+    _check_out(topk_idx, "topk_idx", (T, K), torch.int64, dev)
+    E, R = num_experts, num_ranks
+    if layout_out is not None and (layout_out.T, layout_out.K, layout_out.E, layout_out.R) != (T, K, E, R):
+        raise ValueError(f"layout_out was allocated for (T, K, E, R) = "
+                         f"{(layout_out.T, layout_out.K, layout_out.E, layout_out.R)}, got {(T, K, E, R)}")
+    lay = layout_out if layout_out is not None else alloc_layout(T, K, E, R, align, dev)
+    lay.align = align
+    _check_layout(lay, T, K, dev)
+    N_cap = capacity if capacity is not None else worst_case_rows(T, K, E, align)
+    if out is None:
+        x_perm = torch.empty(N_cap, H, dtype=torch.bfloat16, device=dev)
+        r2f = torch.empty(N_cap, dtype=torch.int32, device=dev)
+        f2r = torch.empty(T, K, dtype=torch.int32, device=dev)
+    else:
+        x_perm, r2f, f2r = out
+        _check_out(x_perm, "x_perm", (N_cap, H), torch.bfloat16, dev)
+        _check_out(r2f, "row_to_flat", (N_cap,), torch.int32, dev)
+        _check_out(f2r, "flat_to_row", (T, K), torch.int32, dev)
+    st = status if status is not None else new_status(dev)
+    rc = lib().moe_dispatch(
+        _ptr(x), _ptr(topk_idx), T, K, E, R, H, align, _ptr(lay.tokens_per_expert),
+        _ptr(lay.counts), _ptr(lay.splits), _ptr(lay.tokens_per_rank), _ptr(lay.is_token_in_rank),
+        _ptr(lay.expert_offsets), _ptr(lay.workspace), int(bool(zero_pad)), N_cap, _ptr(x_perm),
+        _ptr(r2f), _ptr(f2r), _ptr(st), _stream(dev))
+    check_rc(rc, "moe_dispatch")
+    return lay, x_perm, r2f, f2r
+
+
 def expert_scale(rows: torch.Tensor, layout: Layout, scales: torch.Tensor,
                  status: torch.Tensor | None = None, out: torch.Tensor | None = None):
     """Stand-in expert: y = bf16_rn(rows * s_e) on real rows, 0 on pad rows."""

@@ -122,6 +122,37 @@ int moe_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E,
                                       stream));
 }
 
+int moe_dispatch(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int R, int H,
+                 int align, int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                 int32_t* tokens_per_rank, uint8_t* is_token_in_rank, int32_t* expert_offsets,
+                 void* workspace, int zero_pad, int64_t N_cap, uint16_t* x_perm,
+                 int32_t* row_to_flat, int32_t* flat_to_row, int32_t* status,
+                 cudaStream_t stream) {
+    NvtxRange range("moe_dispatch");
+    // Every check of both calls, before anything is enqueued.
+    if (!sizes_ok(T, K, E) || R < 1 || R > MOE_MAX_R || E % R || T % R || align < 1 ||
+        !hidden_ok(H) || !ncap_ok(N_cap, T, K))
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)T * K + (int64_t)E * (align - 1) > INT32_MAX) return MOE_ERR_INVALID_ARG;
+    if (!tokens_per_expert || !counts || !splits || !tokens_per_rank || !expert_offsets ||
+        !workspace || !status)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !topk_idx || !is_token_in_rank || !flat_to_row)) return MOE_ERR_INVALID_ARG;
+    if (N_cap > 0 && (!x_perm || !row_to_flat)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(topk_idx, 8) ||
+        !aligned(workspace, 16) || !aligned(tokens_per_expert, 4) || !aligned(counts, 4) ||
+        !aligned(splits, 4) || !aligned(tokens_per_rank, 4) || !aligned(expert_offsets, 4) ||
+        !aligned(row_to_flat, 4) || !aligned(flat_to_row, 4) || !aligned(status, 4))
+        return MOE_ERR_INVALID_ARG;
+    const cudaError_t e = moe::launch_layout(topk_idx, T, K, E, R, align, tokens_per_expert,
+                                             counts, splits, tokens_per_rank, is_token_in_rank,
+                                             expert_offsets, workspace, status, stream);
+    if (e != cudaSuccess) return finish(e);
+    return finish(moe::launch_permute(x, topk_idx, T, K, E, H, expert_offsets, workspace,
+                                      zero_pad, N_cap, x_perm, row_to_flat, flat_to_row, status,
+                                      stream));
+}
+
 int moe_expert_scale(const uint16_t* rows, int64_t N_cap, const int32_t* expert_offsets,
                      const int32_t* tokens_per_expert, int E, int H, const float* scales,
                      uint16_t* out, int32_t* status, cudaStream_t stream) {

@@ -218,6 +218,20 @@ int moe_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E,
                 int64_t N_cap, uint16_t* x_perm, int32_t* row_to_flat, int32_t* flat_to_row,
                 int32_t* status, cudaStream_t stream);
 
+/* The layout and the permute in one call ([DeepEP-272]: the layout, then
+ * the dispatch with its handle): moe_dispatch_layout, then moe_permute on its
+ * outputs, with the arguments, outputs, status bits and errors of both; every
+ * check of both runs before anything is enqueued, so an invalid argument
+ * leaves the stream untouched.  The workspace is filled as by
+ * moe_dispatch_layout and may be passed on to moe_permute_payload and the
+ * other calls that take a layout. */
+int moe_dispatch(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int R, int H,
+                 int align, int32_t* tokens_per_expert, int32_t* counts, int32_t* splits,
+                 int32_t* tokens_per_rank, uint8_t* is_token_in_rank, int32_t* expert_offsets,
+                 void* workspace, int zero_pad, int64_t N_cap, uint16_t* x_perm,
+                 int32_t* row_to_flat, int32_t* flat_to_row, int32_t* status,
+                 cudaStream_t stream);
+
 /* Stand-in expert between dispatch and combine: for each expert e, its real
  * rows [off[e], off[e] + c_e) become bf16_rn(fp32(row) * scales[e]) (the
  * product rounded to fp32, then once to bf16); its pad rows become zero;

@@ -39,8 +39,9 @@ def f32(bits: np.ndarray) -> np.ndarray:
 
 
 def run_gpu(inp: dict, E: int, R: int, align: int, N_cap: int, *, zero_pad=True, validate=True,
-            weights=None, backward=True, device="cuda:0"):
-    """All calls of the path through the binding; returns numpy copies."""
+            weights=None, backward=True, fused=False, device="cuda:0"):
+    """All calls of the path through the binding; returns numpy copies.  With
+    fused, the layout and the permute are one call (moe_dispatch)."""
     from combine_moe_dispatch_03_b200 import api
     dev = torch.device(device)
     x = inp["x"].to(dev)
@@ -50,11 +51,16 @@ def run_gpu(inp: dict, E: int, R: int, align: int, N_cap: int, *, zero_pad=True,
     T, H = x.shape
     K = topk.shape[1]
     st = api.new_status(dev)
-    lay = api.dispatch_layout(topk, E, R, align, status=st)
     xp = fill_bits((N_cap, H), SENTINEL, dev)
     r2f = torch.empty(N_cap, dtype=torch.int32, device=dev)
     f2r = torch.empty(T, K, dtype=torch.int32, device=dev)
-    api.permute(x, topk, lay, capacity=N_cap, zero_pad=zero_pad, status=st, out=(xp, r2f, f2r))
+    if fused:
+        lay, _, _, _ = api.dispatch(x, topk, E, R, align, capacity=N_cap, zero_pad=zero_pad,
+                                    status=st, out=(xp, r2f, f2r))
+    else:
+        lay = api.dispatch_layout(topk, E, R, align, status=st)
+        api.permute(x, topk, lay, capacity=N_cap, zero_pad=zero_pad, status=st,
+                    out=(xp, r2f, f2r))
     y = fill_bits((N_cap, H), SENTINEL, dev)
     api.expert_scale(xp, lay, s, status=st, out=y)
     out = api.combine_weighted(y, f2r, w, row_to_flat=r2f, validate=validate, status=st)

@@ -106,6 +106,24 @@ def test_layout_host_checks(L, kw):
     assert rc == -1
 
 
+@pytest.mark.parametrize("kw", [
+    dict(H=60), dict(xp=A16 + 2), dict(x=A16 + 8), dict(topk=A16 + 4), dict(N=127),
+    dict(K=0), dict(K=33), dict(E=1025), dict(T=-1), dict(ws=0), dict(status=0),   # permute's
+    dict(R=3), dict(T=63), dict(align=0), dict(R=0), dict(R=65), dict(cnt=0),      # layout's
+    dict(ws=A16 + 8), dict(itr=0), dict(f2r=0), dict(r2f=A16 + 2),
+])
+def test_dispatch_host_checks(L, kw):
+    """moe_dispatch runs every check of the layout and of the permute before
+    it enqueues anything."""
+    a = dict(x=A16, topk=A16, T=64, K=2, E=8, R=2, H=64, align=4, cnt=A16, itr=A16, ws=A16,
+             N=128, xp=A16, r2f=A16, f2r=A16, status=A16)
+    a.update(kw)
+    rc = L.moe_dispatch(a["x"], a["topk"], a["T"], a["K"], a["E"], a["R"], a["H"], a["align"],
+                        A16, a["cnt"], A16, A16, a["itr"], A16, a["ws"], 1, a["N"], a["xp"],
+                        a["r2f"], a["f2r"], a["status"], None)
+    assert rc == -1
+
+
 @pytest.mark.parametrize("kw", [dict(wd=2), dict(H=12), dict(out=A16 + 4), dict(w=A16 + 2),
                                 dict(f2r=0), dict(validate=1, r2f=0)])
 def test_combine_host_checks(L, kw):

@@ -5,7 +5,8 @@ the C ABI accepts (logical ranks R, experts per rank, tokens per rank, top_k
 up to the maximum of 32, row widths that end in a partial 4 KB piece, group
 alignments, a buffer larger than the worst case, zero-padded or not, FP32 or
 bf16 router weights, routing by softmax top-k or by independent draws with
-repeated experts), then runs every call of the path forward and backward and
+repeated experts, the layout and the permute as two calls or as one), then
+runs every call of the path forward and backward and
 compares every output with the oracle: bit-exact for the layout, the row
 maps and every row buffer, the stated tolerance (and the oracle's FP32
 slot-order chain, bit-exact) for the combine outputs and gradients.  The
@@ -44,8 +45,8 @@ def test_random_problems_match_oracle():
            K=st.sampled_from([1, 2, 2, 2, 3, 4, 6, 8, 8, 9, 16, 32]),
            hv=st.integers(1, 700), align=st.sampled_from([1, 2, 3, 8, 16, 17, 64, 128, 160]),
            extra=st.sampled_from([0, 0, 1, 37]), zero_pad=st.booleans(), bf16_w=st.booleans(),
-           repeats=st.booleans(), seed=st.integers(0, 2 ** 31 - 1))
-    def case(R, El, Tb, K, hv, align, extra, zero_pad, bf16_w, repeats, seed):
+           repeats=st.booleans(), fused=st.booleans(), seed=st.integers(0, 2 ** 31 - 1))
+    def case(R, El, Tb, K, hv, align, extra, zero_pad, bf16_w, repeats, fused, seed):
         E, T = R * El, R * Tb
         if K > E:
             repeats = True                          # softmax top-k needs K <= E
@@ -58,7 +59,7 @@ def test_random_problems_match_oracle():
             inp = custom_inputs(T, H, E, K, seed=seed)
         N_cap = capacity_rows(T, K, E, align) + extra
         w = inp["weights"].to(torch.bfloat16) if bf16_w else None
-        gpu = run_gpu(inp, E, R, align, N_cap, zero_pad=zero_pad, weights=w)
+        gpu = run_gpu(inp, E, R, align, N_cap, zero_pad=zero_pad, weights=w, fused=fused)
         ref = run_oracle(inp, E, R, align, N_cap, zero_pad=zero_pad, weights=w)
         compare(gpu, ref, bf16_weights=bf16_w)
         assert np.all(gpu["row_to_flat"][int(gpu["expert_offsets"][-1]):] == -1)

@@ -49,6 +49,31 @@ def test_config_full_size(name):
     _check(inp, cfg.E, cfg.R, cfg.align)
 
 
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "qwen3"])
+def test_fused_dispatch_full_size(name):
+    """moe_dispatch (layout and permute in one call): every output against
+    the oracle, and bit-identical to the two separate calls."""
+    cfg = CONFIGS[name]
+    inp = make_inputs(name, with_grad=True)
+    gpu, _ = _check(inp, cfg.E, cfg.R, cfg.align, fused=True)
+    N = capacity_rows(cfg.T, cfg.K, cfg.E, cfg.align)
+    sep = run_gpu(inp, cfg.E, cfg.R, cfg.align, N)
+    for k in ("x_perm", "row_to_flat", "flat_to_row", "expert_offsets", "counts", "splits",
+              "tokens_per_rank", "is_token_in_rank", "out", "grad_x", "grad_w"):
+        np.testing.assert_array_equal(gpu[k], sep[k], err_msg=k)
+
+
+@pytest.mark.parametrize("T,H,E,K,R,align", [
+    (0, 64, 4, 2, 2, 8), (1, 8, 1, 1, 1, 1), (100, 2048, 8, 2, 1, 16), (777, 24, 5, 1, 1, 3),
+    (4000, 2056, 8, 2, 2, 16), (3008, 4104, 1024, 2, 64, 1), (160000, 8, 16, 2, 2, 8),
+    (997, 264, 13, 5, 1, 8),
+])
+def test_fused_dispatch_edge_shapes(T, H, E, K, R, align):
+    inp = custom_inputs(T, H, E, K, seed=T * 5 + K + 1)
+    N_cap = 16 if T == 0 else None
+    _check(inp, E, R, align, N_cap=N_cap, fused=True)
+
+
 def test_tiny_twice_deterministic():
     cfg = CONFIGS["tiny"]
     inp = make_inputs("tiny", with_grad=True)

@@ -27,8 +27,8 @@ class MoEDispatchCombine(torch.autograd.Function):
     def forward(ctx, x, topk_idx, weights, scales, num_experts: int, num_ranks: int = 1,
                 align: int = 1, validate: bool = False):
         status = api.new_status(x.device)
-        lay = api.dispatch_layout(topk_idx, num_experts, num_ranks, align, status=status)
-        x_perm, r2f, f2r = api.permute(x, topk_idx, lay, status=status)
+        lay, x_perm, r2f, f2r = api.dispatch(x, topk_idx, num_experts, num_ranks, align,
+                                             status=status)
         y = api.expert_scale(x_perm, lay, scales, status=status)
         out = api.combine_weighted(y, f2r, weights, row_to_flat=r2f, validate=validate,
                                    status=status)

@@ -39,6 +39,7 @@ def test_random_problems_match_oracle():
     from hypothesis import HealthCheck, given, settings
     from hypothesis import strategies as st
 
+    ran = []
     @settings(max_examples=300, deadline=None, derandomize=True,
               suppress_health_check=list(HealthCheck))
     @given(R=st.sampled_from([1, 1, 2, 3, 4, 8]), El=st.integers(1, 24), Tb=st.integers(0, 500),
@@ -47,6 +48,7 @@ def test_random_problems_match_oracle():
            extra=st.sampled_from([0, 0, 1, 37]), zero_pad=st.booleans(), bf16_w=st.booleans(),
            repeats=st.booleans(), fused=st.booleans(), seed=st.integers(0, 2 ** 31 - 1))
     def case(R, El, Tb, K, hv, align, extra, zero_pad, bf16_w, repeats, fused, seed):
+        ran.append(1)
         E, T = R * El, R * Tb
         if K > E:
             repeats = True                          # softmax top-k needs K <= E
@@ -65,3 +67,4 @@ def test_random_problems_match_oracle():
         assert np.all(gpu["row_to_flat"][int(gpu["expert_offsets"][-1]):] == -1)
 
     case()
+    assert len(ran) >= 50, len(ran)      # the draws really ran

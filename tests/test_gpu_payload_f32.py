@@ -118,9 +118,13 @@ def _grad_w_ok(got, ref, mag, what):
     (200, 128, 64, 12, 1, torch.float32, 623),        # top-12: the any-K kernels
 ])
 def test_fp32_rows_dispatch_restore_backward(T, H, E, K, align, wdtype, seed):
+    _check_fp32(T, H, E, K, align, wdtype, seed)
+
+
+def _check_fp32(T, H, E, K, align, wdtype, seed, topk=None):
     api = _api()
     dev = torch.device("cuda:0")
-    inp = custom_inputs(T, H, E, K, seed=seed)
+    inp = custom_inputs(T, H, E, K, seed=seed, topk_idx=topk)
     g = torch.Generator().manual_seed(seed + 1)
     x = torch.randn(T, H, generator=g)
     grad = torch.randn(T, H, generator=g)
@@ -158,6 +162,87 @@ def test_fp32_rows_dispatch_restore_backward(T, H, E, K, align, wdtype, seed):
         assert (np.abs(gw.float().cpu().numpy() - bw["grad_w"]) <= lim).all()
     u = orc.combine_f32(bw["grad_rows"], pm["flat_to_row"], None)
     np.testing.assert_array_equal(unit.cpu().numpy(), u["seq"])
+
+
+def test_random_payloads_match_oracle():
+    """Hypothesis (derandomised): opaque payload rows of random byte widths
+    (16-byte units, rows ending in a partial 4 KB piece), with or without a
+    per-token aux payload of a few 4-byte words, any fan-out up to 32 with
+    repeated experts, padded or not: rows, aux rows and both maps bit-exact
+    against the oracle, and rows past the padded total untouched."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+    api = _api()
+    dev = torch.device("cuda:0")
+
+    ran = []
+    @settings(max_examples=150, deadline=None, derandomize=True,
+              suppress_health_check=list(HealthCheck))
+    @given(E=st.integers(1, 64), T=st.integers(0, 700), K=st.sampled_from([1, 2, 3, 4, 8, 9, 32]),
+           m=st.integers(1, 400), aux_words=st.sampled_from([0, 0, 1, 2, 3, 7]),
+           align=st.sampled_from([1, 2, 16, 33, 128]), zero_pad=st.booleans(),
+           seed=st.integers(0, 2 ** 31 - 1))
+    def case(E, T, K, m, aux_words, align, zero_pad, seed):
+        ran.append(1)
+        m = max(1, min(m, 2_000_000 // (16 * max(1, T * K))))
+        g = torch.Generator().manual_seed(seed)
+        x = torch.randint(0, 256, (T, 16 * m), dtype=torch.uint8, generator=g)
+        topk = torch.randint(0, E, (T, K), generator=g)
+        aux = torch.randn(T, aux_words, generator=g) if aux_words else None
+        N_cap = capacity_rows(T, K, E, align) + 3
+        st_ = api.new_status(dev)
+        lay = _layout(topk, E, align, dev, st_)
+        xp = torch.full((N_cap, 16 * m), SENT8, dtype=torch.uint8, device=dev)
+        ap = torch.full((N_cap, aux_words), 7.0, device=dev) if aux_words else None
+        r2f = torch.empty(N_cap, dtype=torch.int32, device=dev)
+        f2r = torch.empty(T, K, dtype=torch.int32, device=dev)
+        api.permute_payload(x.to(dev), topk.to(dev), lay,
+                            aux=aux.to(dev) if aux_words else None, capacity=N_cap,
+                            zero_pad=zero_pad, status=st_, out=(xp, ap, r2f, f2r))
+        torch.cuda.synchronize()
+        assert int(st_.item()) == 0
+        ref = orc.permute_payload(x.numpy(), topk.numpy(), E, lay.expert_offsets.cpu().numpy(),
+                                  N_cap, aux=aux.numpy() if aux_words else None,
+                                  zero_pad=zero_pad,
+                                  x_perm_init=np.full((N_cap, 16 * m), SENT8, np.uint8),
+                                  aux_perm_init=(np.full((N_cap, aux_words), 7.0, np.float32)
+                                                 if aux_words else None))
+        assert ref["status"] == 0
+        np.testing.assert_array_equal(r2f.cpu().numpy(), ref["row_to_flat"])
+        np.testing.assert_array_equal(f2r.cpu().numpy(), ref["flat_to_row"])
+        assert np.array_equal(xp.cpu().numpy(), ref["x_perm"])
+        if aux_words:
+            np.testing.assert_array_equal(ap.cpu().numpy().view(np.uint32),
+                                          ref["aux_perm"].view(np.uint32))
+
+    case()
+    assert len(ran) >= 50, len(ran)      # the draws really ran
+
+
+def test_random_fp32_rows_match_oracle():
+    """Hypothesis (derandomised): fp32 rows through dispatch, the restore,
+    its backward and the unit-weight restore, at random shapes, fan-outs
+    (the slot-major kernels up to K = 8, the any-K ones above), router
+    dtypes and routings with repeated experts; the bars of the fixed cases
+    above."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+
+    ran = []
+    @settings(max_examples=60, deadline=None, derandomize=True,
+              suppress_health_check=list(HealthCheck))
+    @given(E=st.integers(1, 48), T=st.integers(1, 500), K=st.sampled_from([1, 2, 3, 5, 8, 9, 13]),
+           m=st.integers(1, 300), align=st.sampled_from([1, 4, 16, 17]), bf16_w=st.booleans(),
+           seed=st.integers(0, 2 ** 31 - 1))
+    def case(E, T, K, m, align, bf16_w, seed):
+        ran.append(1)
+        m = max(1, min(m, 400_000 // (4 * T * K)))
+        topk = torch.randint(0, E, (T, K), generator=torch.Generator().manual_seed(seed))
+        _check_fp32(T, 4 * m, E, K, align, torch.bfloat16 if bf16_w else torch.float32, seed,
+                    topk=topk)
+
+    case()
+    assert len(ran) >= 50, len(ran)      # the draws really ran
 
 
 def test_payload_argument_errors():

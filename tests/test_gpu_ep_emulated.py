@@ -281,3 +281,42 @@ def _run_direct(inp, R, E, align):
     out_ref = api.combine_weighted(api.expert_scale(xp, lay, sc, status=st), f2r, w, status=st)
     assert torch.equal(_i16(torch.cat(outs)), _i16(out_ref))
     api.check_status(st)
+
+
+# ------------------------------------------------------- random problems ---
+
+def test_ep_random_problems_emulated():
+    """Hypothesis (derandomised): random rank counts, experts per rank,
+    tokens per rank, top_k (softmax top-k or independent draws with repeated
+    experts; any-K kernels above 8), row widths and alignments, through the
+    all-to-all form or the direct form, emulated on one GPU; every value
+    checked against the oracle as in the fixed cases above (plans, grouped
+    and expert rows, claims, planted coverage faults, outputs)."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+
+    ran = []
+
+    @settings(max_examples=40, deadline=None, derandomize=True,
+              suppress_health_check=list(HealthCheck))
+    @given(R=st.sampled_from([1, 2, 3, 4, 8]), El=st.integers(1, 12), extra_t=st.integers(1, 150),
+           K=st.sampled_from([1, 2, 3, 4, 8, 10]), hv=st.integers(1, 300),
+           align=st.sampled_from([1, 4, 16, 17]), repeats=st.booleans(), direct=st.booleans(),
+           seed=st.integers(0, 2 ** 31 - 1))
+    def case(R, El, extra_t, K, hv, align, repeats, direct, seed):
+        ran.append(1)
+        E = R * El
+        Tb = R + extra_t                  # > R tokens per rank: some owner repeats in rank 0
+        T = R * Tb
+        if K > E:
+            repeats = True                # softmax top-k needs K <= E
+        H = 8 * max(1, min(hv, 1_500_000 // (8 * T * K)))
+        if repeats:
+            topk = torch.randint(0, E, (T, K), generator=torch.Generator().manual_seed(seed))
+            inp = custom_inputs(T, H, E, K, seed=seed, topk_idx=topk)
+        else:
+            inp = custom_inputs(T, H, E, K, seed=seed)
+        (_run_direct if direct else _run_emulated)(inp, R, E, align)
+
+    case()
+    assert len(ran) >= 30, len(ran)       # the draws really ran

@@ -211,7 +211,9 @@ int moe_dispatch_layout_noalloc(const int64_t* topk_idx, int T, int K, int E, in
  * Out: x_perm [N_cap,H] bf16, row_to_flat [N_cap] int32, flat_to_row [T,K]
  *      int32 (-1 for an assignment that was not placed).
  * Status: MOE_ST_CAPACITY (rows >= N_cap are not written),
- *         MOE_ST_EXPERT_OOR, MOE_ST_LAYOUT_MISMATCH (nothing written).
+ *         MOE_ST_EXPERT_OOR, MOE_ST_LAYOUT_MISMATCH (nothing written),
+ *         MOE_ST_TIMEOUT (K <= 2: a bounded wait on the kernel's own
+ *         shared-memory copies gave up; outputs undefined).
  * Errors: MOE_ERR_INVALID_ARG as for the layout, or N_cap < A. */
 int moe_permute(const uint16_t* x, const int64_t* topk_idx, int T, int K, int E, int H,
                 const int32_t* expert_offsets, const void* workspace, int zero_pad,

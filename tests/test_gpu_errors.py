@@ -211,6 +211,12 @@ def test_python_layer_refuses_mismatched_shapes():
         api.expert_scale(xp, lay, torch.ones(7, device=dev))
     with pytest.raises(ValueError):                     # reused layout of other sizes
         api.dispatch_layout(topk[:32].contiguous(), 8, 2, 4, out=lay)
+    with pytest.raises(ValueError):                     # one-call dispatch: topk rows != x rows
+        api.dispatch(x[:32].contiguous(), topk, 8, 2, 4)
+    with pytest.raises(ValueError):                     # ... a layout of other sizes
+        api.dispatch(x[:32].contiguous(), topk[:32].contiguous(), 8, 2, 4, layout_out=lay)
+    with pytest.raises(ValueError):                     # ... an undersized row map
+        api.dispatch(x, topk, 8, 2, 4, out=(xp, r2f[:10], f2r))
     torch.cuda.synchronize()
     assert st.item() == 0
 
